@@ -1,0 +1,118 @@
+"""The five synthetic packs the path is tested and measured on, and their inputs.
+
+Each sample is ``(n_text, H_lat, W_lat, frames)``: ``n_text`` text tokens, then
+``frames`` latent grids of ``H_lat`` rows x ``W_lat`` columns, flattened row
+major. Grid sizes follow the 16x latent downsampling of the tokenizer
+(Mage-Flow paper summary, "Mage-VAE": 1024^2 -> 64x64); the resolutions and
+aspect ratios (512^2 to 2048^2, 4:1) follow its "Native-Resolution MMDiT"
+section and the 512-2048 / 4:1 range it quotes. No dataset stands behind these
+inputs: every value is drawn by :mod:`packed_attention_b200.synth`.
+
+Only shapes and value distributions live here; nothing in this module computes
+any part of the attention.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import synth
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    samples: tuple  # of (n_text, H_lat, W_lat, frames)
+    heads: int
+    head_dim: int
+    seed: int
+    token_budget: int = 0
+    # (first_token, last_token_exclusive, sigma): tokens drawn N(0, sigma) instead of N(0, 1)
+    sigma_ranges: tuple = ()
+    # fraction of raw K token rows (all heads) multiplied by outlier_scale
+    outlier_frac: float = 0.0
+    outlier_scale: float = 1.0
+    eps: float = 1e-6
+    notes: str = field(default="", compare=False)
+
+    @property
+    def seg_lens(self):
+        return [nt + f * h * w for (nt, h, w, f) in self.samples]
+
+    @property
+    def total_tokens(self) -> int:
+        return sum(self.seg_lens)
+
+    @property
+    def sum_L2(self) -> int:
+        return sum(L * L for L in self.seg_lens)
+
+    @property
+    def flops(self) -> int:
+        """Algorithmic FLOPs of the attention: 4 * H * d * sum_i L_i^2."""
+        return 4 * self.heads * self.head_dim * self.sum_L2
+
+    def with_heads(self, heads: int) -> "Workload":
+        return Workload(self.name + f"_h{heads}", self.samples, heads, self.head_dim, self.seed,
+                        self.token_budget, self.sigma_ranges, self.outlier_frac, self.outlier_scale,
+                        self.eps, self.notes)
+
+
+WORKLOADS = {
+    0: Workload("tiny_pack", ((16, 8, 8, 1), (8, 4, 16, 1)), heads=2, head_dim=64, seed=0,
+                notes="two samples: 16 text + 8x8 grid, 8 text + 4x16 grid"),
+    1: Workload("uniform_512sq", ((128, 32, 32, 1),) * 4, heads=24, head_dim=128, seed=1,
+                notes="4 x (128 text + 32x32 grid) = 4608 tokens"),
+    2: Workload("mixed_native_res",
+                ((77, 32, 32, 1), (200, 48, 64, 1), (256, 64, 64, 1),
+                 (40, 16, 64, 1), (128, 64, 48, 1), (99, 40, 40, 1)),
+                heads=24, head_dim=128, seed=2, token_budget=15400,
+                notes="six native-resolution samples, 14,688 tokens under a 15,400-token budget"),
+    3: Workload("edit_1024sq", ((512, 64, 64, 2),), heads=24, head_dim=128, seed=3,
+                sigma_ranges=((512 + 4096, 512 + 2 * 4096, 0.5),),
+                notes="512 text + 64x64 target + 64x64 reference grid (same positions), 8704 tokens"),
+    4: Workload("hires_2048sq_4to1", ((512, 128, 128, 1), (256, 32, 128, 1)), heads=24,
+                head_dim=128, seed=4, outlier_frac=0.01, outlier_scale=8.0,
+                notes="2048^2 sample (16,896 tokens) + 4:1 sample (4,352 tokens); 1% of K rows x8"),
+}
+
+
+def make_inputs(w: Workload):
+    """bf16 bit patterns (uint16) for q, k, v ``[T, H, d]`` and the four gammas.
+
+    Gammas are returned as fp32 arrays holding bf16-representable values
+    ``bf16(1 + 0.1 z)``. Returns a dict of numpy arrays.
+    """
+    T, H, d = w.total_tokens, w.heads, w.head_dim
+    n = T * H * d
+    sig = np.ones(T, dtype=np.float64)
+    for lo, hi, s in w.sigma_ranges:
+        sig[lo:hi] = s
+    out = {}
+    for name, stream in (("q", synth.STREAM_Q), ("k", synth.STREAM_K), ("v", synth.STREAM_V)):
+        z = synth.normals(w.seed, stream, n).reshape(T, H, d)
+        if w.sigma_ranges:
+            z *= sig[:, None, None]
+        out[name] = synth.f64_to_bf16_bits(z)
+    if w.outlier_frac > 0:
+        n_rows = int(round(w.outlier_frac * T))
+        rows = synth.choose_rows(w.seed, synth.STREAM_OUTLIER_ROWS, T, n_rows)
+        kv = synth.bf16_bits_to_f64(out["k"][rows]) * w.outlier_scale
+        out["k"][rows] = synth.f64_to_bf16_bits(kv)
+        out["outlier_rows"] = rows
+    for name, stream in (("g_q_text", synth.STREAM_GQ_TEXT), ("g_q_img", synth.STREAM_GQ_IMG),
+                         ("g_k_text", synth.STREAM_GK_TEXT), ("g_k_img", synth.STREAM_GK_IMG)):
+        g = 1.0 + 0.1 * synth.normals(w.seed, stream, d)
+        out[name] = synth.bf16_bits_to_f64(synth.f64_to_bf16_bits(g)).astype(np.float32)
+    return out
+
+
+def random_pack(rng: np.random.Generator, n_samples: int, max_text: int, max_side: int,
+                max_frames: int = 1):
+    """A random list of samples for small parity and edge-case packs."""
+    out = []
+    for _ in range(n_samples):
+        out.append((int(rng.integers(0, max_text + 1)), int(rng.integers(1, max_side + 1)),
+                    int(rng.integers(1, max_side + 1)), int(rng.integers(1, max_frames + 1))))
+    return tuple(out)
