@@ -1,0 +1,349 @@
+"""Benchmark of the packed joint text+image attention forward on B200.
+
+One step = one pass of the whole hot path over one synthetic pack: the
+QK-RMSNorm + 2D-RoPE prologue and the block-diagonal attention, launched
+through the C ABI on the current stream. Default workload: the
+high-resolution pack (a 2048^2 sample of 16,896 tokens and a 4:1 sample of
+4,352 tokens, 24 heads, head_dim 128, 1% of key rows x8).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl native|reference]
+
+Under torchrun every rank runs its own replica of the workload (the pack's
+(sample, head) units are independent; there is no collective on the data
+path) and rank 0 prints one JSON line with the whole-job throughput.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "packed joint-attention TFLOP/s and tokens/s on 1 B200; % of dense-BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows
+                                   if r[3].replace(".", "").isdigit()) if rows else None}
+
+
+def oracle_sample_rows(w, rng, n_blocks, block=64):
+    """Rows for a bounded oracle sample: blocks of `block` consecutive tokens of
+    one head, drawn in proportion to the tokens of each sample."""
+    lens = np.array(w.seg_lens)
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    rows = []
+    flops = 0
+    for _ in range(n_blocks):
+        s = int(rng.choice(len(lens), p=lens / lens.sum()))
+        h = int(rng.integers(0, w.heads))
+        b = int(rng.integers(0, max(1, lens[s] - block + 1)))
+        toks = np.arange(starts[s] + b, starts[s] + min(b + block, lens[s]))
+        rows.append(toks * w.heads + h)
+        flops += 4 * w.head_dim * int(lens[s]) * len(toks)
+    return np.unique(np.concatenate(rows)), flops
+
+
+def oracle_throughput(w, inp, seconds, seed=0):
+    """The fp64 oracle, as it stands, on all host cores: TFLOP/s on sampled rows."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    cores = os.cpu_count() or 1
+    rows, flops = oracle_sample_rows(w, rng, max(1, cores))
+    t0 = time.perf_counter()
+    oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
+    dt = time.perf_counter() - t0
+    n_blocks = max(cores, int(cores * seconds / max(dt, 1e-3)))
+    rows, flops = oracle_sample_rows(w, rng, n_blocks)
+    t0 = time.perf_counter()
+    oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, cores, f"{len(rows)} of {w.total_tokens * w.heads} (token, head) " \
+        f"query rows in 64-token blocks, {flops / 1e9:.1f} GFLOP, {dt:.1f} s"
+
+
+def run_reference(args, w):
+    """Reference arm: the fp64 oracle on host cores, one bounded sample per step."""
+    from packed_attention_b200.workloads import make_inputs
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = make_inputs(w)
+    cores = os.cpu_count() or 1
+    import oracle
+    rng = np.random.default_rng(1234)
+    budget = 150.0 / max(1, args.steps + args.warmup)  # seconds of CPU work per step
+    # calibrate block count per step
+    rows, _ = oracle_sample_rows(w, rng, cores)
+    t0 = time.perf_counter()
+    oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
+    per_block = (time.perf_counter() - t0) / cores
+    n_blocks = max(1, int(budget / max(per_block, 1e-4)))
+    for _ in range(args.warmup):
+        rows, _ = oracle_sample_rows(w, rng, n_blocks)
+        oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
+    total_flops, total_t = 0, 0.0
+    for _ in range(args.steps):
+        rows, fl = oracle_sample_rows(w, rng, n_blocks)
+        t0 = time.perf_counter()
+        oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
+        total_t += time.perf_counter() - t0
+        total_flops += fl
+    value = total_flops / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "total_tokens": w.total_tokens, "heads": w.heads,
+                   "head_dim": w.head_dim, "samples": [list(s) for s in w.samples]},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {n_blocks} blocks of 64 query rows of one head, "
+                                   f"fp64 oracle on {cores} threads"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    from packed_attention_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[args.config]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import packed_attention_b200 as pa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    inp = make_inputs(w)
+    T, H, d = w.total_tokens, w.heads, w.head_dim
+    t = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).to(dev)
+         for n in ("q", "k", "v")}
+    t.update({n: torch.from_numpy(inp[n]).to(dev) for n in pa.GAMMA_NAMES})
+    plan = pa.PackedPlan(w.samples, H, d, w.token_budget, device=dev)
+    ws = plan.new_workspace()
+    out = torch.empty_like(t["q"])
+    stream = torch.cuda.current_stream()
+
+    def step(e0=None, e1=None, e2=None):
+        if e0 is not None:
+            e0.record(stream)
+        pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=w.eps)
+        if e1 is not None:
+            e1.record(stream)
+        pa.packed_attention(t["v"], plan, ws, out)
+        if e2 is not None:
+            e2.record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if pa.device_error() != 0:
+        raise RuntimeError("kernel reported a device-side error during warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    start.record(stream)
+    for i in range(K):
+        step(*evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    if pa.device_error() != 0:
+        raise RuntimeError("kernel reported a device-side error in the timed region")
+
+    total_ms = start.elapsed_time(end)
+    pro_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    att_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    timing = torch.tensor([total_ms, pro_ms, att_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(timing, op=dist.ReduceOp.MAX)
+    total_ms, pro_ms, att_ms = timing.tolist()
+
+    # ---- end to end through the public API on host buffers (copies timed) ----
+    host = {n: t[n].cpu().pin_memory() for n in ("q", "k", "v", *pa.GAMMA_NAMES)}
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    bufs = {}
+    for _ in range(2):
+        pa.joint_attention_host(host["q"], host["k"], host["v"], host, plan, eps=w.eps,
+                                out_host=out_host, device_buffers=bufs)
+    torch.cuda.synchronize()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_s.record(stream)
+    for _ in range(args.e2e_steps):
+        pa.joint_attention_host(host["q"], host["k"], host["v"], host, plan, eps=w.eps,
+                                out_host=out_host, device_buffers=bufs)
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = torch.tensor([e_s.elapsed_time(e_e) / args.e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    flops = w.flops
+    step_s = total_ms / K / 1e3
+    value = flops * world / step_s / 1e12
+    tokens_per_s = T * world / step_s
+    att_tflops = flops / (att_ms / 1e3) / 1e12
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    peak_burst = float(peaks["bf16_tflops"])
+    pro_bytes = 8 * T * H * d
+    pro_gbs = pro_bytes / (pro_ms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        v_cpu, cores, sample = oracle_throughput(w, inp, args.cpu_seconds)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    h2d = sum(host[n].numel() * host[n].element_size() for n in host)
+    d2h = out_host.numel() * out_host.element_size()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": w.name, "samples": [list(s) for s in w.samples], "total_tokens": T,
+            "heads": H, "head_dim": d, "sum_L2": w.sum_L2, "gflop_per_step": flops / 1e9,
+            "parallelism": "independent replicas" if world > 1 else "single gpu",
+            "l2": f"inputs q,k,v = {3 * T * H * d * 2 / 1e6:.0f} MB > 126 MB L2 (not flushed)",
+        },
+        "tokens_per_s": tokens_per_s,
+        "pct_of_peak": 100.0 * value / world / peak_sus,
+        "roofline": {
+            "kernel": "packed_attention_kernel", "bound": "tensor", "achieved": att_tflops,
+            "peak": peak_sus, "unit": "TFLOP/s", "frac": att_tflops / peak_sus,
+            "peak_kind": f"{peak_src} bf16 dense, sustained",
+            "frac_of_burst_peak": att_tflops / peak_burst, "traffic": None,
+            "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_ms,
+        },
+        "prologue": {
+            "kernel": "qk_prologue_kernel", "bound": "hbm", "achieved": pro_gbs, "peak": hbm,
+            "unit": "GB/s", "frac": pro_gbs / hbm, "algorithmic_bytes_per_launch": pro_bytes,
+            "avg_launch_ms": pro_ms,
+        },
+        "cpu_baseline": cpu,
+        "e2e": {"value": flops * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

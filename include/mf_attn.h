@@ -1,0 +1,187 @@
+/*
+ * mf_attn.h -- C ABI of the packed joint text+image attention forward
+ * (the attention hot path of Mage-Flow's Native-Resolution MMDiT), for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation. Images of different resolutions and aspect ratios are
+ * flattened to latent token sequences and packed, with their variable-length
+ * text tokens, into one buffer without padding; attention runs inside each
+ * sample only, which per-sample cumulative offsets (cu_seqlens) describe
+ * [Mage-Flow paper summary, "Native-Resolution MMDiT (NR-MMDiT)";
+ * video overview, 00:03:16-00:04:03]. Text and image streams are normalised
+ * with separate parameters before the joint self-attention [same section:
+ * modality-specific normalization], and image tokens carry per-sample 2D
+ * rotary position embeddings [video overview, 00:03:16; capabilities page,
+ * "Key Capabilities"].
+ *
+ * Readings this library adopts where the pages give no formula:
+ *  - Sample layout: n_text text tokens, then `frames` latent grids of
+ *    grid_h x grid_w tokens, each flattened row-major. An editing sample has
+ *    frames = 2 (target, then reference); every frame uses the same grid
+ *    positions.
+ *  - Normalisation: RMSNorm over head_dim for each (token, head) of q and k,
+ *    x * rsqrt(mean(x^2) + eps) * gamma, with four gamma vectors of length
+ *    head_dim (q/k x text/image) shared by all heads. V is untouched.
+ *  - 2D RoPE, after the norm, image tokens only: grid row r rotates dims
+ *    [0, d/2), grid column c rotates dims [d/2, d), in adjacent pairs
+ *    (2j, 2j+1) by pos * 10000^(-2j/(d/2)). Text tokens are not rotated.
+ *  - Attention: non-causal softmax(q_hat k_hat^T * scale) v within a sample.
+ *
+ * Conventions for every entry point:
+ *  - Errors are returned as mf_status; nothing aborts, throws or prints.
+ *  - Device entry points are asynchronous on the caller's stream (`stream` is
+ *    a cudaStream_t; NULL is the legacy default stream) and allocate nothing,
+ *    so they can be captured in a CUDA graph.
+ *  - All device pointers are owned by the caller; inputs are never written.
+ *  - Launch failures return MF_ERR_CUDA. A fault the kernels detect while
+ *    running (a pipeline wait that exceeded its time limit) is recorded on
+ *    the device and reported by mf_get_device_error().
+ */
+#ifndef MF_ATTN_H
+#define MF_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MF_OK = 0,
+  MF_ERR_INVALID_ARG = -1, /* NULL pointer, negative or inconsistent size      */
+  MF_ERR_UNSUPPORTED = -2, /* head_dim not in {64, 128}                         */
+  MF_ERR_ALIGNMENT = -3,   /* a device pointer is not 16-byte aligned           */
+  MF_ERR_WORKSPACE = -4,   /* workspace_bytes < mf_workspace_bytes(...)         */
+  MF_ERR_BUDGET = -5,      /* total tokens exceed the pack's token budget       */
+  MF_ERR_CUDA = -6,        /* a CUDA runtime or driver call failed              */
+  MF_ERR_TIMEOUT = -7      /* a kernel pipeline wait ran out of time            */
+} mf_status;
+
+/* One packed sample: tokens [start, start + len) of the pack. 24 bytes. */
+typedef struct {
+  int32_t start;
+  int32_t len;    /* n_text + frames * grid_h * grid_w */
+  int32_t n_text;
+  int32_t grid_h; /* latent rows    */
+  int32_t grid_w; /* latent columns */
+  int32_t frames;
+} mf_segment;
+
+/* One unit of attention work: query rows
+ * [segs[seg].start + q_tile * MF_TILE_M, min(+MF_TILE_M, segment end)) of head `head`,
+ * attending over all kv_len keys of the sample. 16 bytes. */
+typedef struct {
+  int32_t seg;
+  int32_t head;
+  int32_t q_tile;
+  int32_t kv_len;
+} mf_work_item;
+
+#define MF_TILE_M 128 /* query rows per work item */
+#define MF_TILE_N 128 /* keys per pipeline step   */
+
+/* ABI version of this header (incremented on any change of signature). */
+int32_t mf_abi_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* mf_status_string(mf_status status);
+
+/*
+ * mf_pack_plan -- host only; builds the per-sample layout and the work list.
+ * [Mage-Flow summary, "Native-Resolution MMDiT": packing under a fixed token
+ *  budget with per-sample cumulative offsets; video overview, 00:04:03: zero
+ *  padding.]
+ *
+ * Inputs (host arrays of n_samples entries each):
+ *   n_text[i] >= 0, grid_h[i] >= 1, grid_w[i] >= 1, frames[i] >= 1
+ *   (frames == NULL means 1 for every sample). heads >= 1.
+ *   head_dim must be 64 or 128 (checked here so a plan never describes work
+ *   the kernels cannot run). token_budget <= 0 means no budget.
+ * Outputs (host, caller-owned; each may be NULL to skip it):
+ *   cu_seqlens [n_samples + 1]   prefix sums of the sample lengths, int32
+ *   segs       [n_samples]       mf_segment per sample
+ *   work       [*n_work]         work items ordered longest sample first
+ *                                (ties: sample index, then head, then q_tile)
+ *   n_work, total_tokens         scalars (may be NULL)
+ * Two-call convention: call with work == NULL to learn *n_work, then again
+ * with *n_work set to the capacity of `work` (at least the count returned);
+ * *n_work then receives the count written. A non-NULL `work` needs a non-NULL
+ * n_work. The sum of the lengths is exact: no rounding of segments to tiles,
+ * no padding tokens.
+ * Errors: MF_ERR_INVALID_ARG for a bad count, size or NULL input array, or a
+ * total that does not fit int32; MF_ERR_UNSUPPORTED for head_dim;
+ * MF_ERR_BUDGET when the total exceeds token_budget (> 0).
+ */
+mf_status mf_pack_plan(int32_t n_samples, const int32_t* n_text, const int32_t* grid_h,
+                       const int32_t* grid_w, const int32_t* frames, int32_t heads,
+                       int32_t head_dim, int64_t token_budget, int32_t* cu_seqlens,
+                       mf_segment* segs, mf_work_item* work, int32_t* n_work,
+                       int32_t* total_tokens);
+
+/*
+ * Bytes of device workspace mf_joint_attn_fwd needs: the normalised, rotated
+ * q_hat and k_hat ([T, H, d] bf16 each) plus a small control block.
+ * Returns 0 for invalid sizes.
+ */
+size_t mf_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim);
+
+/*
+ * mf_qk_prologue -- stage 1 of mf_joint_attn_fwd, exposed for measurement.
+ * For every token and head, RMSNorm q and k with the gamma of the token's
+ * modality and rotate image tokens by their grid position (see the readings
+ * above); writes q_hat and k_hat (bf16, [T, H, d]) into the workspace and
+ * resets the work-list counter the attention stage pops from.
+ *   q, k           bf16 [total_tokens, heads, head_dim], contiguous, 16-B aligned
+ *   g_q_text ...   fp32 [head_dim] each, device
+ *   cu_seqlens_dev int32 [n_samples + 1], device, from mf_pack_plan
+ *   segs_dev       mf_segment [n_samples], device, from mf_pack_plan
+ *   eps            added to the mean square (e.g. 1e-6), must be >= 0
+ *   workspace      device, >= mf_workspace_bytes(...), 256-B aligned
+ */
+mf_status mf_qk_prologue(const void* q, const void* k, const float* g_q_text,
+                         const float* g_q_img, const float* g_k_text, const float* g_k_img,
+                         const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                         int32_t n_samples, int32_t total_tokens, int32_t heads,
+                         int32_t head_dim, float eps, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * mf_packed_attention -- stage 2 of mf_joint_attn_fwd, exposed for
+ * measurement: block-diagonal softmax attention of q_hat, k_hat (read from
+ * the workspace that mf_qk_prologue filled) and v, on tensor cores.
+ *   v              bf16 [total_tokens, heads, head_dim], contiguous, 16-B aligned
+ *   work_dev       mf_work_item [n_work], device, from mf_pack_plan
+ *   softmax_scale  <= 0 selects 1/sqrt(head_dim)
+ *   out            bf16 [total_tokens, heads, head_dim], 16-B aligned, must not
+ *                  overlap q, k, v or the workspace
+ */
+mf_status mf_packed_attention(const void* v, const mf_segment* segs_dev, int32_t n_samples,
+                              const mf_work_item* work_dev, int32_t n_work, int32_t total_tokens,
+                              int32_t heads, int32_t head_dim, float softmax_scale, void* out,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mf_joint_attn_fwd -- the whole forward: mf_qk_prologue then
+ * mf_packed_attention on `stream`. Arguments as described above.
+ */
+mf_status mf_joint_attn_fwd(const void* q, const void* k, const void* v, const float* g_q_text,
+                            const float* g_q_img, const float* g_k_text, const float* g_k_img,
+                            const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                            int32_t n_samples, const mf_work_item* work_dev, int32_t n_work,
+                            int32_t total_tokens, int32_t heads, int32_t head_dim, float eps,
+                            float softmax_scale, void* out, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the error the kernels
+ * recorded on the current device since the last call (MF_OK if none,
+ * MF_ERR_TIMEOUT if a pipeline wait ran out of time and the kernel gave up).
+ */
+mf_status mf_get_device_error(void* stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* MF_ATTN_H */

@@ -1,0 +1,20 @@
+"""B200-native packed joint text+image attention forward (Mage-Flow NR-MMDiT hot path).
+
+The compute lives in ``libmfattn.so`` (hand-written sm_100a CUDA behind the C ABI
+in ``include/mf_attn.h``); this package marshals torch tensors into it.
+Importing the package does not load the library; the first call does, and
+raises if the library has not been built.
+"""
+from ._native import MfError, MF_TILE_M, MF_TILE_N, pack_plan, workspace_bytes  # noqa: F401
+
+__all__ = ["MfError", "MF_TILE_M", "MF_TILE_N", "pack_plan", "workspace_bytes",
+           "PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
+           "packed_attention", "workspace_views", "device_error"]
+
+
+def __getattr__(name):
+    if name in ("PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
+                "packed_attention", "workspace_views", "device_error", "GAMMA_NAMES"):
+        from . import api
+        return getattr(api, name)
+    raise AttributeError(name)

@@ -1,0 +1,159 @@
+"""PyTorch-facing API: device memory and streams come from torch, all compute
+runs in libmfattn's CUDA kernels through the C ABI (``include/mf_attn.h``).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native
+from ._native import check, lib
+
+GAMMA_NAMES = ("g_q_text", "g_q_img", "g_k_text", "g_k_img")
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream_handle(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class PackedPlan:
+    """Host plan from ``mf_pack_plan`` plus its device copies."""
+
+    def __init__(self, samples, heads: int, head_dim: int, token_budget: int = 0,
+                 device: torch.device | str = "cuda"):
+        host = _native.pack_plan(samples, heads, head_dim, token_budget)
+        self.host = host
+        self.samples = [tuple(s) + (1,) * (4 - len(s)) for s in samples]
+        self.n_samples = host["n_samples"]
+        self.total_tokens = host["total_tokens"]
+        self.heads = heads
+        self.head_dim = head_dim
+        self.n_work = int(host["work"].shape[0])
+        self.device = torch.device(device)
+        self.cu_seqlens = torch.from_numpy(host["cu_seqlens"]).to(self.device)
+        self.segs = torch.from_numpy(host["segs"]).to(self.device)
+        self.work = torch.from_numpy(host["work"]).to(self.device)
+
+    @property
+    def seg_lens(self):
+        return [int(x) for x in self.host["segs"][:, 1]]
+
+    @property
+    def flops(self) -> int:
+        return 4 * self.heads * self.head_dim * sum(L * L for L in self.seg_lens)
+
+    def workspace_bytes(self) -> int:
+        return _native.workspace_bytes(self.total_tokens, self.heads, self.head_dim)
+
+    def new_workspace(self) -> torch.Tensor:
+        return torch.empty(self.workspace_bytes(), dtype=torch.uint8, device=self.device)
+
+
+def workspace_views(ws: torch.Tensor, plan: PackedPlan):
+    """(q_hat, k_hat) bf16 [T, H, d] views into a workspace filled by the prologue."""
+    n = plan.total_tokens * plan.heads * plan.head_dim
+    tensor_bytes = (2 * n + 255) // 256 * 256
+    qh = ws[:2 * n].view(torch.bfloat16).view(plan.total_tokens, plan.heads, plan.head_dim)
+    kh = ws[tensor_bytes:tensor_bytes + 2 * n].view(torch.bfloat16).view(
+        plan.total_tokens, plan.heads, plan.head_dim)
+    return qh, kh
+
+
+def _check_qkv(plan: PackedPlan, *ts):
+    shape = (plan.total_tokens, plan.heads, plan.head_dim)
+    for t in ts:
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous() \
+                or not t.is_cuda:
+            raise ValueError(f"expected a contiguous CUDA bf16 tensor of shape {shape}")
+
+
+def _gammas(gammas, plan):
+    gs = [gammas[n] for n in GAMMA_NAMES]
+    for g in gs:
+        if g.dtype != torch.float32 or tuple(g.shape) != (plan.head_dim,) or not g.is_cuda:
+            raise ValueError("gammas must be CUDA float32 tensors of shape [head_dim]")
+    return gs
+
+
+def qk_prologue(q, k, gammas, plan: PackedPlan, workspace: torch.Tensor, eps: float = 1e-6,
+                stream=None):
+    _check_qkv(plan, q, k)
+    gs = _gammas(gammas, plan)
+    check("mf_qk_prologue", lib().mf_qk_prologue(
+        _ptr(q), _ptr(k), *[_ptr(g) for g in gs], _ptr(plan.cu_seqlens), _ptr(plan.segs),
+        plan.n_samples, plan.total_tokens, plan.heads, plan.head_dim, float(eps), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)))
+
+
+def packed_attention(v, plan: PackedPlan, workspace: torch.Tensor, out: torch.Tensor,
+                     softmax_scale: float = 0.0, stream=None):
+    _check_qkv(plan, v, out)
+    check("mf_packed_attention", lib().mf_packed_attention(
+        _ptr(v), _ptr(plan.segs), plan.n_samples, _ptr(plan.work), plan.n_work, plan.total_tokens,
+        plan.heads, plan.head_dim, float(softmax_scale), _ptr(out), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)))
+
+
+def joint_attention(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
+                    softmax_scale: float = 0.0, out: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Packed joint text+image attention forward on device tensors.
+
+    q, k, v: bf16 [T, H, d] CUDA tensors; gammas: dict of the four fp32 [d]
+    CUDA tensors (g_q_text, g_q_img, g_k_text, g_k_img). Returns bf16 [T, H, d].
+    """
+    _check_qkv(plan, q, k, v)
+    gs = _gammas(gammas, plan)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_qkv(plan, out)
+    if workspace is None:
+        workspace = plan.new_workspace()
+    check("mf_joint_attn_fwd", lib().mf_joint_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), *[_ptr(g) for g in gs], _ptr(plan.cu_seqlens),
+        _ptr(plan.segs), plan.n_samples, _ptr(plan.work), plan.n_work, plan.total_tokens,
+        plan.heads, plan.head_dim, float(eps), float(softmax_scale), _ptr(out), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)))
+    return out
+
+
+def joint_attention_host(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
+                         softmax_scale: float = 0.0, out_host: torch.Tensor | None = None,
+                         device_buffers: dict | None = None, stream=None) -> torch.Tensor:
+    """Same forward on HOST tensors: copies inputs to the device, runs, copies the
+    result back into ``out_host`` (pinned host memory makes the copies async).
+
+    ``device_buffers`` may hold preallocated q, k, v, out, workspace and gamma
+    tensors to reuse across calls.
+    """
+    b = device_buffers if device_buffers is not None else {}
+    dev = plan.device
+    for name, src in (("q", q), ("k", k), ("v", v)):
+        if name not in b:
+            b[name] = torch.empty(src.shape, dtype=src.dtype, device=dev)
+        b[name].copy_(src, non_blocking=True)
+    for name in GAMMA_NAMES:
+        if name not in b:
+            b[name] = torch.empty(gammas[name].shape, dtype=torch.float32, device=dev)
+        b[name].copy_(gammas[name], non_blocking=True)
+    if "out" not in b:
+        b["out"] = torch.empty_like(b["q"])
+    if "workspace" not in b:
+        b["workspace"] = plan.new_workspace()
+    joint_attention(b["q"], b["k"], b["v"], {n: b[n] for n in GAMMA_NAMES}, plan, eps,
+                    softmax_scale, out=b["out"], workspace=b["workspace"], stream=stream)
+    if out_host is None:
+        out_host = torch.empty(b["out"].shape, dtype=b["out"].dtype, pin_memory=True)
+    out_host.copy_(b["out"], non_blocking=True)
+    return out_host
+
+
+def device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the kernels' error code."""
+    return int(lib().mf_get_device_error(_stream_handle(stream)))

@@ -1,0 +1,223 @@
+// C-ABI entry points of libmfattn: argument checks, workspace layout, TMA
+// descriptor encoding and kernel launches on the caller's stream. All device
+// code of the library lives in this translation unit (the kernels are in the
+// included headers).
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/mf_attn.h"
+#include "packed_attention.cuh"
+#include "qk_prologue.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kCtlBytes = 256;
+constexpr int kMaxDevices = 64;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WorkspaceLayout {
+  size_t q_hat;
+  size_t k_hat;
+  size_t ctl;
+  size_t total;
+};
+
+bool layout(int32_t total_tokens, int32_t heads, int32_t head_dim, WorkspaceLayout* w) {
+  if (total_tokens < 1 || heads < 1 || (head_dim != 64 && head_dim != 128)) return false;
+  const size_t tensor = round_up(static_cast<size_t>(total_tokens) * heads * head_dim * 2, kAlign);
+  w->q_hat = 0;
+  w->k_hat = tensor;
+  w->ctl = 2 * tensor;
+  w->total = 2 * tensor + kCtlBytes;
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [T, H, d] bf16 viewed as a 3-D tensor (d, H, T); boxes of 64 dims x 1 head
+// x 128 tokens with the 128-byte swizzle the MMA descriptors expect. Boxes
+// that run past T are zero-filled.
+bool encode_thd(CUtensorMap* map, const void* base, int32_t T, int32_t H, int32_t D) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(mf::kBlockM)};
+  cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+bool prepare_attention_kernel() {
+  static std::once_flag once[kMaxDevices];
+  static bool ok[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::call_once(once[dev], [dev] {
+    ok[dev] = cudaFuncSetAttribute(mf::packed_attention_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   mf::AttnConfig<D>::kSmemBytes) == cudaSuccess;
+  });
+  return ok[dev];
+}
+
+}  // namespace
+
+extern "C" size_t mf_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim) {
+  WorkspaceLayout w;
+  return layout(total_tokens, heads, head_dim, &w) ? w.total : 0;
+}
+
+extern "C" mf_status mf_qk_prologue(const void* q, const void* k, const float* g_q_text,
+                                    const float* g_q_img, const float* g_k_text,
+                                    const float* g_k_img, const int32_t* cu_seqlens_dev,
+                                    const mf_segment* segs_dev, int32_t n_samples,
+                                    int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                    float eps, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
+  WorkspaceLayout w;
+  if (!layout(total_tokens, heads, head_dim, &w) || n_samples < 1 || !(eps >= 0.0f) ||
+      !std::isfinite(eps))
+    return MF_ERR_INVALID_ARG;
+  if (!q || !k || !g_q_text || !g_q_img || !g_k_text || !g_k_img || !cu_seqlens_dev || !segs_dev ||
+      !workspace)
+    return MF_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MF_ERR_ALIGNMENT;
+  if (workspace_bytes < w.total) return MF_ERR_WORKSPACE;
+  const size_t bytes = static_cast<size_t>(total_tokens) * heads * head_dim * 2;
+  if (overlaps(workspace, w.total, q, bytes) || overlaps(workspace, w.total, k, bytes))
+    return MF_ERR_INVALID_ARG;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int vec_per_row = head_dim / 8;
+  const int tok_per_block = mf::kPrologueThreads / vec_per_row;
+  const unsigned grid = static_cast<unsigned>((total_tokens + tok_per_block - 1) / tok_per_block);
+  auto* counter = reinterpret_cast<int32_t*>(ws + w.ctl);
+  if (head_dim == 128) {
+    mf::qk_prologue_kernel<128><<<grid, mf::kPrologueThreads, 0, s>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
+        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps,
+        reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat), counter);
+  } else {
+    mf::qk_prologue_kernel<64><<<grid, mf::kPrologueThreads, 0, s>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
+        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps,
+        reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat), counter);
+  }
+  return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
+}
+
+extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_dev,
+                                         int32_t n_samples, const mf_work_item* work_dev,
+                                         int32_t n_work, int32_t total_tokens, int32_t heads,
+                                         int32_t head_dim, float softmax_scale, void* out,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
+  WorkspaceLayout w;
+  if (!layout(total_tokens, heads, head_dim, &w) || n_samples < 1 || n_work < 1)
+    return MF_ERR_INVALID_ARG;
+  if (!v || !segs_dev || !work_dev || !out || !workspace) return MF_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MF_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MF_ERR_ALIGNMENT;
+  if (workspace_bytes < w.total) return MF_ERR_WORKSPACE;
+  const size_t bytes = static_cast<size_t>(total_tokens) * heads * head_dim * 2;
+  if (overlaps(out, bytes, v, bytes) || overlaps(out, bytes, workspace, w.total))
+    return MF_ERR_INVALID_ARG;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUtensorMap tq, tk, tv;
+  if (!encode_thd(&tq, ws + w.q_hat, total_tokens, heads, head_dim) ||
+      !encode_thd(&tk, ws + w.k_hat, total_tokens, heads, head_dim) ||
+      !encode_thd(&tv, v, total_tokens, heads, head_dim))
+    return MF_ERR_CUDA;
+
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  mf::AttnParams prm;
+  prm.segs = segs_dev;
+  prm.work = work_dev;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.heads = heads;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128) {
+    if (!prepare_attention_kernel<128>()) return MF_ERR_CUDA;
+    mf::packed_attention_kernel<128>
+        <<<n_work, mf::kAttnThreads, mf::AttnConfig<128>::kSmemBytes, s>>>(tq, tk, tv, prm);
+  } else {
+    if (!prepare_attention_kernel<64>()) return MF_ERR_CUDA;
+    mf::packed_attention_kernel<64>
+        <<<n_work, mf::kAttnThreads, mf::AttnConfig<64>::kSmemBytes, s>>>(tq, tk, tv, prm);
+  }
+  return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
+}
+
+extern "C" mf_status mf_joint_attn_fwd(const void* q, const void* k, const void* v,
+                                       const float* g_q_text, const float* g_q_img,
+                                       const float* g_k_text, const float* g_k_img,
+                                       const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                                       int32_t n_samples, const mf_work_item* work_dev,
+                                       int32_t n_work, int32_t total_tokens, int32_t heads,
+                                       int32_t head_dim, float eps, float softmax_scale, void* out,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  // Check everything the second stage needs before launching the first.
+  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
+  if (!v || !work_dev || !out || n_work < 1 || !std::isfinite(softmax_scale))
+    return MF_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(out)) return MF_ERR_ALIGNMENT;
+  const size_t bytes = static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * heads * head_dim * 2;
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes)) return MF_ERR_INVALID_ARG;
+  mf_status st = mf_qk_prologue(q, k, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev,
+                                segs_dev, n_samples, total_tokens, heads, head_dim, eps, workspace,
+                                workspace_bytes, stream);
+  if (st != MF_OK) return st;
+  return mf_packed_attention(v, segs_dev, n_samples, work_dev, n_work, total_tokens, heads,
+                             head_dim, softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+extern "C" mf_status mf_get_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MF_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, mf::g_device_error, sizeof v) != cudaSuccess) return MF_ERR_CUDA;
+  if (v != 0) {
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(mf::g_device_error, &zero, sizeof zero) != cudaSuccess)
+      return MF_ERR_CUDA;
+  }
+  return static_cast<mf_status>(v);
+}

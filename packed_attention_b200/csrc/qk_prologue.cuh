@@ -1,0 +1,150 @@
+// Stage 1: modality-selected QK-RMSNorm + per-sample 2D RoPE.
+//
+// [Mage-Flow paper summary, "Native-Resolution MMDiT (NR-MMDiT)":
+//  modality-specific normalization before joint self-attention; video
+//  overview, 00:03:16, and capabilities page, "Key Capabilities": per-sample
+//  2D rotary embeddings on the latent grid.]
+//
+// For every token t and head h, and X in {q, k}:
+//   x_hat = x * rsqrt(mean(x^2) + eps) * gamma_{X, modality(t)}
+// then, for image tokens at grid (r, c), dims [0, d/2) rotate pairwise by
+// r * theta_j and dims [d/2, d) by c * theta_j, theta_j = 10000^(-2j/(d/2)).
+// Text tokens are not rotated. All arithmetic in fp32, one bf16 rounding.
+//
+// HBM-bound: it reads q and k and writes q_hat and k_hat once (8 * T * H * d
+// bytes). Layout of the work: a group of d/8 threads owns one token and
+// loops over its heads; each thread holds 8 consecutive dims (one 16-byte
+// vector) of q and of k, so a warp reads and writes whole 256-byte rows.
+// The token's position, gammas and the 4 (cos, sin) pairs a thread needs are
+// computed once per token and reused for all heads and for both q and k.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "../../include/mf_attn.h"
+
+namespace mf {
+
+constexpr int kPrologueThreads = 256;
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
+  uint4 v;
+  v.x = pack_bf16x2(y[0], y[1]);
+  v.y = pack_bf16x2(y[2], y[3]);
+  v.z = pack_bf16x2(y[4], y[5]);
+  v.w = pack_bf16x2(y[6], y[7]);
+  return v;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
+    const uint4* __restrict__ q, const uint4* __restrict__ k, const float* __restrict__ gq_text,
+    const float* __restrict__ gq_img, const float* __restrict__ gk_text,
+    const float* __restrict__ gk_img, const int32_t* __restrict__ cu_seqlens,
+    const mf_segment* __restrict__ segs, int n_samples, int total_tokens, int heads, float eps,
+    uint4* __restrict__ q_hat, uint4* __restrict__ k_hat, int32_t* __restrict__ work_counter) {
+  constexpr int kVecPerRow = D / 8;                          // 16-byte vectors per row
+  constexpr int kTokPerBlock = kPrologueThreads / kVecPerRow;
+  constexpr int kHalf = D / 2;
+
+  if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
+
+  const int vec = threadIdx.x % kVecPerRow;
+  const int t_raw = blockIdx.x * kTokPerBlock + threadIdx.x / kVecPerRow;
+  // Threads past the last token compute on a valid token (so every lane of
+  // the warp takes part in the shuffles) and store nothing.
+  const bool active = t_raw < total_tokens;
+  const int t = active ? t_raw : total_tokens - 1;
+
+  // Sample that holds t: the last i with cu_seqlens[i] <= t.
+  int lo = 0, hi = n_samples;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(cu_seqlens + mid) <= t) lo = mid; else hi = mid;
+  }
+  const int start = __ldg(&segs[lo].start);
+  const int n_text = __ldg(&segs[lo].n_text);
+  const int gw = __ldg(&segs[lo].grid_w);
+  const int hw = __ldg(&segs[lo].grid_h) * gw;
+  const int j = t - start;
+  const bool is_text = j < n_text;
+
+  const int e0 = vec * 8;  // first dim this thread owns
+  float cs[4], sn[4];
+  if (is_text) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { cs[i] = 1.0f; sn[i] = 0.0f; }
+  } else {
+    const int p = (j - n_text) % hw;  // every frame of a sample shares the grid positions
+    const int axis = e0 >= kHalf;     // 0: grid row, 1: grid column
+    const float pos = static_cast<float>(axis ? p % gw : p / gw);
+    const int pair0 = (e0 - axis * kHalf) / 2;
+    // theta_j = 10000^(-2j/half) = 2^(-(2j/half) * log2(10000))
+    constexpr float kLog2Base = 13.287712379549449f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float theta = exp2f(-(2.0f * (pair0 + i) / kHalf) * kLog2Base);
+      sincosf(pos * theta, &sn[i], &cs[i]);
+    }
+  }
+
+  float gq[8], gk[8];
+  {
+    const float* gqs = is_text ? gq_text : gq_img;
+    const float* gks = is_text ? gk_text : gk_img;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      gq[i] = __ldg(gqs + e0 + i);
+      gk[i] = __ldg(gks + e0 + i);
+    }
+  }
+
+  const float inv_d = 1.0f / D;
+  const size_t row0 = static_cast<size_t>(t) * heads * kVecPerRow + vec;
+#pragma unroll 2
+  for (int h = 0; h < heads; ++h) {
+    const size_t idx = row0 + static_cast<size_t>(h) * kVecPerRow;
+    float xq[8], xk[8];
+    unpack8(__ldg(q + idx), xq);
+    unpack8(__ldg(k + idx), xk);
+    float ssq = 0.f, ssk = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ssq = fmaf(xq[i], xq[i], ssq);
+      ssk = fmaf(xk[i], xk[i], ssk);
+    }
+#pragma unroll
+    for (int o = kVecPerRow / 2; o > 0; o >>= 1) {
+      ssq += __shfl_xor_sync(0xffffffffu, ssq, o, kVecPerRow);
+      ssk += __shfl_xor_sync(0xffffffffu, ssk, o, kVecPerRow);
+    }
+    const float rq = rsqrtf(fmaf(ssq, inv_d, eps));
+    const float rk = rsqrtf(fmaf(ssk, inv_d, eps));
+    float yq[8], yk[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float qa = xq[2 * i] * rq * gq[2 * i], qb = xq[2 * i + 1] * rq * gq[2 * i + 1];
+      const float ka = xk[2 * i] * rk * gk[2 * i], kb = xk[2 * i + 1] * rk * gk[2 * i + 1];
+      yq[2 * i] = qa * cs[i] - qb * sn[i];
+      yq[2 * i + 1] = qa * sn[i] + qb * cs[i];
+      yk[2 * i] = ka * cs[i] - kb * sn[i];
+      yk[2 * i + 1] = ka * sn[i] + kb * cs[i];
+    }
+    if (active) {
+      q_hat[idx] = pack8(yq);
+      k_hat[idx] = pack8(yk);
+    }
+  }
+}
+
+}  // namespace mf

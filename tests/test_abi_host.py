@@ -1,0 +1,157 @@
+"""Host-side tests of libmfattn: exported symbols, the pack planner and argument
+checks. No GPU is touched: every call here returns before any CUDA work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import packed_attention_b200 as pa
+from packed_attention_b200 import _native
+from packed_attention_b200.build import build
+from packed_attention_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _native.lib()
+
+
+def header_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(mf_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert "mf_pack_plan" in names and "mf_joint_attn_fwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    # and the binding covers exactly the declared API
+    assert sorted(_native.SIGNATURES) == names
+
+
+def test_status_strings(lib):
+    assert lib.mf_abi_version() == 1
+    for code, name in _native.STATUS.items():
+        assert lib.mf_status_string(code).decode() == name
+
+
+def test_struct_sizes_match_header():
+    assert ctypes.sizeof(_native.Segment) == 24
+    assert ctypes.sizeof(_native.WorkItem) == 16
+
+
+@pytest.mark.parametrize("cfg,cu", [
+    (0, [0, 80, 152]),
+    (1, [0, 1152, 2304, 3456, 4608]),
+    (2, [0, 1101, 4373, 8725, 9789, 12989, 14688]),
+    (3, [0, 8704]),
+    (4, [0, 16896, 21248]),
+])
+def test_plan_offsets_by_hand(lib, cfg, cu):
+    w = WORKLOADS[cfg]
+    p = pa.pack_plan(w.samples, w.heads, w.head_dim, w.token_budget)
+    assert p["cu_seqlens"].tolist() == cu
+    assert p["total_tokens"] == cu[-1]  # no padding, no rounding to tiles
+    segs = p["segs"]
+    for i, (nt, gh, gw, fr) in enumerate(w.samples):
+        assert segs[i].tolist() == [cu[i], cu[i + 1] - cu[i], nt, gh, gw, fr]
+
+
+@pytest.mark.parametrize("cfg,n_work", [(0, 4), (1, 864), (2, 2808), (3, 1632), (4, 3984)])
+def test_plan_work_list(lib, cfg, n_work):
+    w = WORKLOADS[cfg]
+    p = pa.pack_plan(w.samples, w.heads, w.head_dim, w.token_budget)
+    work = p["work"]
+    assert work.shape == (n_work, 4)
+    lens = p["segs"][:, 1]
+    # every (segment, head, q_tile) exactly once
+    want = {(s, h, t) for s in range(len(lens)) for h in range(w.heads)
+            for t in range((lens[s] + 127) // 128)}
+    got = {tuple(x) for x in work[:, :3].tolist()}
+    assert got == want and len(got) == n_work
+    # kv_len is the segment length; longest first, ties by sample index then head, q_tile
+    assert np.array_equal(work[:, 3], lens[work[:, 0]])
+    keys = [(-int(L), int(s), int(h), int(t)) for s, h, t, L in work.tolist()]
+    assert keys == sorted(keys)
+
+
+def test_plan_budget_and_validation(lib):
+    w = WORKLOADS[2]
+    assert pa.pack_plan(w.samples, 24, 128, 15400)["total_tokens"] == 14688
+    with pytest.raises(pa.MfError) as e:
+        pa.pack_plan(w.samples, 24, 128, 14687)
+    assert e.value.status == -5
+    for bad in ([(1, 0, 4, 1)], [(-1, 2, 2, 1)], [(0, 2, 2, 0)]):
+        with pytest.raises(pa.MfError) as e:
+            pa.pack_plan(bad, 2, 64)
+        assert e.value.status == -1
+    with pytest.raises(pa.MfError) as e:
+        pa.pack_plan([(1, 2, 2, 1)], 2, 96)
+    assert e.value.status == -2
+    with pytest.raises(pa.MfError):  # total beyond int32
+        pa.pack_plan([(0, 46341, 46341, 1)], 1, 64)
+    with pytest.raises(pa.MfError):
+        pa.pack_plan([(0, 1, 1, 1)], 0, 64)
+
+
+def test_plan_two_call_capacity(lib):
+    n_text = (ctypes.c_int32 * 1)(5)
+    gh = (ctypes.c_int32 * 1)(3)
+    gw = (ctypes.c_int32 * 1)(100)
+    n_work = ctypes.c_int32(0)
+    assert lib.mf_pack_plan(1, n_text, gh, gw, None, 2, 64, 0, None, None, None,
+                            ctypes.byref(n_work), None) == 0
+    assert n_work.value == 2 * 3
+    small = (ctypes.c_int32 * 8)()
+    n_work.value = 1  # capacity too small
+    assert lib.mf_pack_plan(1, n_text, gh, gw, None, 2, 64, 0, None, None, small,
+                            ctypes.byref(n_work), None) == -1
+    assert lib.mf_pack_plan(1, n_text, gh, gw, None, 2, 64, 0, None, None, small, None, None) == -1
+
+
+def test_workspace_size(lib):
+    assert pa.workspace_bytes(152, 2, 64) == 2 * ((152 * 2 * 64 * 2 + 255) // 256 * 256) + 256
+    assert pa.workspace_bytes(0, 2, 64) == 0
+    assert pa.workspace_bytes(10, 2, 96) == 0
+
+
+def _fwd(lib, **over):
+    """mf_joint_attn_fwd with fake (never dereferenced) pointers."""
+    a = dict(q=0x10000, k=0x20000, v=0x30000, gqt=0x40000, gqi=0x40100, gkt=0x40200,
+             gki=0x40300, cu=0x50000, segs=0x60000, n=2, work=0x70000, n_work=4, T=152, H=2,
+             d=64, eps=1e-6, scale=0.0, out=0x80000, ws=0x100000, ws_bytes=1 << 20)
+    a.update(over)
+    P = ctypes.c_void_p
+    return lib.mf_joint_attn_fwd(P(a["q"]), P(a["k"]), P(a["v"]), P(a["gqt"]), P(a["gqi"]),
+                                 P(a["gkt"]), P(a["gki"]), P(a["cu"]), P(a["segs"]), a["n"],
+                                 P(a["work"]), a["n_work"], a["T"], a["H"], a["d"], a["eps"],
+                                 a["scale"], P(a["out"]), P(a["ws"]), a["ws_bytes"], None)
+
+
+def test_forward_argument_checks(lib):
+    assert _fwd(lib, d=96) == -2
+    assert _fwd(lib, q=0x10008) == -3
+    assert _fwd(lib, v=0x30004) == -3
+    assert _fwd(lib, out=0x80002) == -3
+    assert _fwd(lib, ws=0x100010) == -3
+    assert _fwd(lib, ws_bytes=100) == -4
+    assert _fwd(lib, q=0) == -1
+    assert _fwd(lib, work=0) == -1
+    assert _fwd(lib, n_work=0) == -1
+    assert _fwd(lib, T=0) == -1
+    assert _fwd(lib, eps=-1.0) == -1
+    assert _fwd(lib, eps=float("nan")) == -1
+    assert _fwd(lib, scale=float("inf")) == -1
+    assert _fwd(lib, out=0x10000) == -1        # out aliases q
+    assert _fwd(lib, ws=0x10000 - 0x100) == -1  # workspace overlaps q

@@ -1,0 +1,203 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bar: max-abs error <= 2e-2 and relative RMS error <= 5e-3 over the compared
+elements (bf16 output, fp32 accumulation); the prologue's q_hat / k_hat
+within one bf16 rounding of the oracle. Small packs are compared element by
+element in full; the five full-size packs run in the same launch
+configuration the benchmark times and are compared on sampled rows (every
+segment's first and last rows, tile boundaries, ragged tails and random
+rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import packed_attention_b200 as pa
+from packed_attention_b200 import synth
+from packed_attention_b200.workloads import WORKLOADS, Workload, make_inputs, random_pack
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_RMS = 5e-3
+
+
+def to_dev(inp, dev):
+    t = {}
+    for name in ("q", "k", "v"):
+        t[name] = torch.from_numpy(inp[name].view(np.int16)).view(torch.bfloat16).to(dev)
+    for name in pa.GAMMA_NAMES:
+        t[name] = torch.from_numpy(inp[name]).to(dev)
+    return t
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def errors(got, ref):
+    diff = got - ref
+    max_abs = float(np.max(np.abs(diff)))
+    rel_rms = float(np.sqrt(np.mean(diff ** 2)) / np.sqrt(np.mean(ref ** 2)))
+    return max_abs, rel_rms
+
+
+def run_gpu(w: Workload, inp, dev, out=None):
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=dev)
+    t = to_dev(inp, dev)
+    out = pa.joint_attention(t["q"], t["k"], t["v"], t, plan, eps=w.eps, out=out)
+    assert pa.device_error() == 0
+    return plan, t, out
+
+
+def sample_rows(w: Workload, rng, n_random=256):
+    """Flat row indices token * H + head: segment edges, tile edges, tails, random."""
+    T, H = w.total_tokens, w.heads
+    toks = set()
+    start = 0
+    for L in w.seg_lens:
+        end = start + L
+        for t in (start, start + 1, end - 2, end - 1):
+            if start <= t < end:
+                toks.add(t)
+        for b in range(start + 127, end, 128):
+            toks.update({b, min(b + 1, end - 1)})
+        last = start + (L - 1) // 128 * 128  # first row of the ragged tail tile
+        toks.update(range(last, min(last + 3, end)))
+        start = end
+    toks = np.array(sorted(toks), dtype=np.int64)
+    heads_e = rng.integers(0, H, size=len(toks))
+    rows = set((toks * H + heads_e).tolist())
+    rows.update(rng.integers(0, T * H, size=n_random).tolist())
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+# ------------------------------------------------------------- prologue ---
+
+@pytest.mark.parametrize("cfg,heads", [(0, None), (2, 2), (3, 1)])
+def test_prologue_matches_oracle(cuda_device, cfg, heads):
+    w = WORKLOADS[cfg] if heads is None else WORKLOADS[cfg].with_heads(heads)
+    inp = make_inputs(w)
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=cuda_device)
+    t = to_dev(inp, cuda_device)
+    ws = plan.new_workspace()
+    pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=w.eps)
+    qh, kh = pa.workspace_views(ws, plan)
+    for got, x, gt, gi in ((qh, "q", "g_q_text", "g_q_img"), (kh, "k", "g_k_text", "g_k_img")):
+        ref = oracle.qk_prologue(inp[x], w.samples, inp[gt], inp[gi], eps=w.eps)
+        g = bf16_to_f64(got)
+        # fp32 arithmetic rounded once to bf16: within one bf16 ulp (2^-7 relative).
+        bound = 2.0 ** -7 * np.abs(ref) + 1e-6
+        bad = np.abs(g - ref) > bound
+        assert not bad.any(), f"{bad.sum()} of {bad.size} {x}_hat elements off by more than 1 ulp"
+        # and at most 0.5 ulp plus fp32 noise for the vast majority
+        assert np.mean(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6) > 0.99
+
+
+# ------------------------------------------------------- small packs, full ---
+
+SMALL_PACKS = [
+    ("tiny_pack", WORKLOADS[0]),
+    ("ragged_d128", Workload("ragged_d128", ((77, 12, 20, 1), (0, 9, 15, 1), (5, 1, 1, 1),
+                                             (200, 8, 8, 2)), heads=3, head_dim=128, seed=11)),
+    ("ragged_d64", Workload("ragged_d64", ((13, 10, 13, 1), (128, 1, 1, 1), (0, 16, 8, 1)),
+                            heads=2, head_dim=64, seed=12)),
+    ("tile_edges", Workload("tile_edges", ((0, 1, 1, 1), (0, 1, 127, 1), (0, 1, 128, 1),
+                                           (0, 1, 129, 1), (1, 16, 16, 1), (0, 1, 257, 1)),
+                            heads=2, head_dim=128, seed=13)),
+    ("config2_shapes_h1", WORKLOADS[2].with_heads(1)),
+]
+
+
+@pytest.mark.parametrize("name,w", SMALL_PACKS, ids=[n for n, _ in SMALL_PACKS])
+def test_small_pack_full_compare(cuda_device, name, w):
+    inp = make_inputs(w)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps)
+    got = bf16_to_f64(out)
+    assert np.all(np.isfinite(got))
+    max_abs, rel_rms = errors(got, ref)
+    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
+
+
+@pytest.mark.parametrize("trial", range(4))
+def test_random_packs_full_compare(cuda_device, trial):
+    rng = np.random.default_rng(500 + trial)
+    samples = random_pack(rng, int(rng.integers(1, 7)), 300, 24, 2)
+    w = Workload(f"random_{trial}", samples, heads=int(rng.integers(1, 4)),
+                 head_dim=(64, 128)[trial % 2], seed=600 + trial)
+    inp = make_inputs(w)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps)
+    max_abs, rel_rms = errors(bf16_to_f64(out), ref)
+    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
+
+
+# ------------------------------------------------ full-size packs, sampled ---
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
+def test_full_size_config_sampled_rows(cuda_device, cfg):
+    w = WORKLOADS[cfg]
+    inp = make_inputs(w)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    got_all = bf16_to_f64(out)
+    assert np.all(np.isfinite(got_all))
+    rng = np.random.default_rng(cfg)
+    rows = sample_rows(w, rng)
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
+    got = got_all.reshape(-1, w.head_dim)[rows]
+    max_abs, rel_rms = errors(got, ref)
+    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
+
+
+# --------------------------------------------------------------- hygiene ---
+
+def test_canary_rows_untouched_and_deterministic(cuda_device):
+    w = SMALL_PACKS[1][1]
+    inp = make_inputs(w)
+    T, H, d = w.total_tokens, w.heads, w.head_dim
+    guard = 200
+    buf = torch.full(((T + 2 * guard) * H * d,), -1000.0, dtype=torch.bfloat16, device=cuda_device)
+    out = buf[guard * H * d:(guard + T) * H * d].view(T, H, d)
+    _, _, out = run_gpu(w, inp, cuda_device, out=out)
+    first = out.clone()
+    torch.cuda.synchronize()
+    pre, post = buf[:guard * H * d], buf[(guard + T) * H * d:]
+    assert torch.all(pre == -1000.0) and torch.all(post == -1000.0)
+    _, _, out = run_gpu(w, inp, cuda_device, out=out)
+    assert torch.equal(first.view(torch.int16), out.view(torch.int16))
+
+
+def test_host_buffer_path_matches_device_path(cuda_device):
+    w = SMALL_PACKS[2][1]
+    inp = make_inputs(w)
+    plan, t, out = run_gpu(w, inp, cuda_device)
+    host = {n: t[n].cpu().pin_memory() for n in ("q", "k", "v", *pa.GAMMA_NAMES)}
+    res = pa.joint_attention_host(host["q"], host["k"], host["v"], host, plan, eps=w.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(res.view(torch.int16), out.cpu().view(torch.int16))
+
+
+def test_key_outliers_are_harmless(cuda_device):
+    # Config 4's recipe (1% of raw K rows x8) on a small pack: parity holds.
+    w = Workload("outliers", ((64, 12, 12, 1), (30, 6, 24, 1)), heads=2, head_dim=128, seed=21,
+                 outlier_frac=0.01, outlier_scale=8.0)
+    inp = make_inputs(w)
+    assert len(inp["outlier_rows"]) == round(0.01 * w.total_tokens)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps)
+    max_abs, rel_rms = errors(bf16_to_f64(out), ref)
+    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS
+
+
+def test_explicit_softmax_scale(cuda_device):
+    w = Workload("scaled", ((10, 8, 9, 1), (3, 5, 5, 1)), heads=2, head_dim=64, seed=22)
+    inp = make_inputs(w)
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, device=cuda_device)
+    t = to_dev(inp, cuda_device)
+    for scale in (0.05, 0.3):
+        out = pa.joint_attention(t["q"], t["k"], t["v"], t, plan, eps=w.eps, softmax_scale=scale)
+        ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, scale=scale)
+        max_abs, rel_rms = errors(bf16_to_f64(out), ref)
+        assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (scale, max_abs, rel_rms)
