@@ -87,14 +87,21 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
   } else {
     const int p = (j - n_text) % hw;  // every frame of a sample shares the grid positions
     const int axis = e0 >= kHalf;     // 0: grid row, 1: grid column
-    const float pos = static_cast<float>(axis ? p % gw : p / gw);
+    const int pos = axis ? p % gw : p / gw;
     const int pair0 = (e0 - axis * kHalf) / 2;
-    // theta_j = 10000^(-2j/half) = 2^(-(2j/half) * log2(10000))
-    constexpr float kLog2Base = 13.287712379549449f;
+    // theta_j = 10000^(-2j/half) = 2^(-(2j/half) * log2(10000)). The angle
+    // pos * theta_j is formed and reduced to [-pi, pi] in fp64 (once per token
+    // and thread), so the fp32 sine and cosine see an argument accurate to
+    // ~1e-7 rad however large the grid position is.
+    constexpr double kLog2Base = 13.287712379549449;
+    constexpr double kTwoPi = 6.283185307179586;
+    constexpr double kInvTwoPi = 0.15915494309189535;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float theta = exp2f(-(2.0f * (pair0 + i) / kHalf) * kLog2Base);
-      sincosf(pos * theta, &sn[i], &cs[i]);
+      const double theta = exp2(-(2.0 * (pair0 + i) / kHalf) * kLog2Base);
+      double ang = static_cast<double>(pos) * theta;
+      ang -= kTwoPi * rint(ang * kInvTwoPi);
+      sincosf(static_cast<float>(ang), &sn[i], &cs[i]);
     }
   }
 

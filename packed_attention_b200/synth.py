@@ -19,6 +19,9 @@ Generator
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -59,11 +62,16 @@ def splitmix64(seed: int, stream: int, n: int, offset: int = 0) -> np.ndarray:
 
 
 def normals(seed: int, stream: int, n: int) -> np.ndarray:
-    """``n`` standard normal fp64 values from stream (seed, stream), Box-Muller."""
+    """``n`` standard normal fp64 values from stream (seed, stream), Box-Muller.
+
+    Chunks are independent (the stream is counter-based), so they are filled
+    by a thread pool; the result does not depend on the thread count.
+    """
     m = (n + 1) // 2
     out = np.empty(2 * m, dtype=np.float64)
     two_pi = 2.0 * np.pi
-    for lo in range(0, m, _CHUNK):
+
+    def fill(lo):
         hi = min(m, lo + _CHUNK)
         w = splitmix64(seed, stream, 2 * (hi - lo), offset=2 * lo)
         u1 = ((w[0::2] >> np.uint64(11)) + np.uint64(1)).astype(np.float64) * 2.0 ** -53
@@ -71,6 +79,13 @@ def normals(seed: int, stream: int, n: int) -> np.ndarray:
         r = np.sqrt(-2.0 * np.log(u1))
         out[2 * lo:2 * hi:2] = r * np.cos(two_pi * u2)
         out[2 * lo + 1:2 * hi:2] = r * np.sin(two_pi * u2)
+
+    starts = list(range(0, m, _CHUNK))
+    if len(starts) > 1:
+        with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
+    elif starts:
+        fill(0)
     return out[:n]
 
 

@@ -13,6 +13,8 @@ any part of the attention.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -94,7 +96,13 @@ def make_inputs(w: Workload):
         z = synth.normals(w.seed, stream, n).reshape(T, H, d)
         if w.sigma_ranges:
             z *= sig[:, None, None]
-        out[name] = synth.f64_to_bf16_bits(z)
+        bits = np.empty(z.shape, dtype=np.uint16)
+        rows = max(1, (1 << 22) // (H * d))
+        with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+            def conv(lo):
+                bits[lo:lo + rows] = synth.f64_to_bf16_bits(z[lo:lo + rows])
+            list(ex.map(conv, range(0, T, rows)))
+        out[name] = bits
     if w.outlier_frac > 0:
         n_rows = int(round(w.outlier_frac * T))
         rows = synth.choose_rows(w.seed, synth.STREAM_OUTLIER_ROWS, T, n_rows)

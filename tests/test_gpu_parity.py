@@ -87,12 +87,14 @@ def test_prologue_matches_oracle(cuda_device, cfg, heads):
     for got, x, gt, gi in ((qh, "q", "g_q_text", "g_q_img"), (kh, "k", "g_k_text", "g_k_img")):
         ref = oracle.qk_prologue(inp[x], w.samples, inp[gt], inp[gi], eps=w.eps)
         g = bf16_to_f64(got)
-        # fp32 arithmetic rounded once to bf16: within one bf16 ulp (2^-7 relative).
-        bound = 2.0 ** -7 * np.abs(ref) + 1e-6
-        bad = np.abs(g - ref) > bound
+        # fp32 arithmetic rounded once to bf16: within one bf16 ulp (2^-7
+        # relative) plus the fp32 error of the norm and rotation, which is
+        # relative to the row's magnitude, not to an element that cancels.
+        slack = 1e-5 * np.max(np.abs(ref), axis=-1, keepdims=True)
+        bad = np.abs(g - ref) > 2.0 ** -7 * np.abs(ref) + slack
         assert not bad.any(), f"{bad.sum()} of {bad.size} {x}_hat elements off by more than 1 ulp"
-        # and at most 0.5 ulp plus fp32 noise for the vast majority
-        assert np.mean(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6) > 0.99
+        # and within half an ulp (2^-8 relative bounds it) for nearly all
+        assert np.mean(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + slack) > 0.999
 
 
 # ------------------------------------------------------- small packs, full ---
