@@ -398,3 +398,24 @@ def test_invalid_samples_rejected():
     assert oracle.total_tokens([(-1, 2, 3, 1)]) == -1
     assert oracle.total_tokens([(1, 2, 3, 0)]) == -1
     assert oracle.total_tokens([(1, 2, 3, 1), (0, 1, 1, 2)]) == 9
+
+
+def test_golden_closed_forms():
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "closed_forms.json")
+    with open(path) as f:
+        gold = json.load(f)
+    for d in (64, 128):
+        x = np.zeros((2, 1, d), dtype=np.uint16)
+        x[:, 0, 2] = ONE_BF16
+        g = np.ones(d, dtype=np.float32)
+        y = oracle.qk_prologue(x, [(0, 2, 1, 1)], g, g, eps=0.0)[1, 0]
+        assert math.atan2(y[3], y[2]) == pytest.approx(gold["rope_theta1"][str(d)], abs=1e-13)
+    for c in gold["rmsnorm_one_hot"]["cases"]:
+        d = c["d"]
+        x = np.zeros((2, 1, d), dtype=np.uint16)
+        x[:, 0, c["m"]] = bits(c["a"])
+        g = np.ones(d, dtype=np.float32)
+        y = oracle.qk_prologue(x, [(1, 1, 1, 1)], g, g, eps=c["eps"])
+        assert y[0, 0, c["m"]] == pytest.approx(c["x_hat_m"], rel=1e-14)
