@@ -174,6 +174,46 @@ mf_status mf_joint_attn_fwd(const void* q, const void* k, const void* v, const f
                             size_t workspace_bytes, void* stream);
 
 /*
+ * mf_joint_attn_fwd_static_scratch -- the same forward for callers that
+ * cannot allocate device memory at all. The paper has no counterpart to this
+ * entry point; it exists for how the library is called, not for the method.
+ *
+ * Who needs it: code that is handed a stream but no allocator -- a plugin
+ * inside a host framework that owns every byte of device memory, a caller in
+ * the middle of a global-mode stream capture (where cudaMalloc is illegal),
+ * or a latency-critical loop that cannot pay for cudaMalloc's implicit device
+ * synchronisation -- and so cannot provide the workspace mf_joint_attn_fwd
+ * asks for.
+ *
+ * Instead of a caller workspace it uses a scratch array of
+ * MF_STATIC_SCRATCH_BYTES bytes that lives in the library itself (a
+ * file-scope device array): every GPU that loads the library holds those
+ * bytes until the process exits. This entry point allocates nothing and
+ * calls no allocating routine. Arguments are those of mf_joint_attn_fwd
+ * without workspace / workspace_bytes; inputs and outputs are still the
+ * caller's.
+ *   - Packs whose scratch need, mf_workspace_bytes(total_tokens, heads,
+ *     head_dim), exceeds MF_STATIC_SCRATCH_BYTES are rejected with
+ *     MF_ERR_WORKSPACE before anything is launched (64 MiB holds q_hat and
+ *     k_hat for up to ~131,000 (token, head) rows at head_dim 128).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - All calls share the one array, and it keeps whatever the last call
+ *     left in it (every call rewrites the parts it reads). Calls whose
+ *     kernels overlap on the GPU -- on two streams, or from two threads --
+ *     race on the array: serialise them.
+ */
+#define MF_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+mf_status mf_joint_attn_fwd_static_scratch(
+    const void* q, const void* k, const void* v, const float* g_q_text, const float* g_q_img,
+    const float* g_k_text, const float* g_k_img, const int32_t* cu_seqlens_dev,
+    const mf_segment* segs_dev, int32_t n_samples, const mf_work_item* work_dev, int32_t n_work,
+    int32_t total_tokens, int32_t heads, int32_t head_dim, float eps, float softmax_scale,
+    void* out, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the error the kernels
  * recorded on the current device since the last call (MF_OK if none,
  * MF_ERR_TIMEOUT if a pipeline wait ran out of time and the kernel gave up).

@@ -59,8 +59,12 @@ SIGNATURES = {
     "mf_packed_attention": (I32, [P, P, I32, P, I32, I32, I32, I32, F32, P, P, SZ, P]),
     "mf_joint_attn_fwd": (I32, [P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, F32, F32, P,
                                 P, SZ, P]),
+    "mf_joint_attn_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32,
+                                               I32, F32, F32, P, P]),
     "mf_get_device_error": (I32, [P]),
 }
+
+MF_STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 def lib():

@@ -25,7 +25,8 @@ NVCC_FLAGS = [
 
 
 def sources():
-    return [os.path.join(CSRC, "mf_attn.cu"), os.path.join(CSRC, "plan.cpp")]
+    return [os.path.join(CSRC, "mf_attn.cu"), os.path.join(CSRC, "static_scratch.cu"),
+            os.path.join(CSRC, "plan.cpp")]
 
 
 def _stale() -> bool:
