@@ -70,7 +70,8 @@ typedef struct {
 
 /* One unit of attention work: query rows
  * [segs[seg].start + q_tile * MF_TILE_M, min(+MF_TILE_M, segment end)) of head `head`,
- * attending over all kv_len keys of the sample. 16 bytes. */
+ * attending over all kv_len keys of the sample. 16 bytes. The kernel splits
+ * an item into two 128-row tensor-core tiles that share every K/V tile. */
 typedef struct {
   int32_t seg;
   int32_t head;
@@ -78,7 +79,7 @@ typedef struct {
   int32_t kv_len;
 } mf_work_item;
 
-#define MF_TILE_M 128 /* query rows per work item */
+#define MF_TILE_M 256 /* query rows per work item */
 #define MF_TILE_N 128 /* keys per pipeline step   */
 
 /* ABI version of this header (incremented on any change of signature). */

@@ -15,7 +15,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmfattn.so")
 
-MF_TILE_M = 128
+MF_TILE_M = 256
 MF_TILE_N = 128
 
 STATUS = {

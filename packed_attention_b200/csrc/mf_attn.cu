@@ -70,12 +70,24 @@ bool encode_thd(CUtensorMap* map, const void* base, int32_t T, int32_t H, int32_
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(T)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
-  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(mf::kBlockM)};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(mf::kSubM)};
   cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                    box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static std::once_flag once[kMaxDevices];
+  static int count[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::call_once(once[dev], [dev] {
+    int c = 0;
+    count[dev] = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? c : 0;
+  });
+  return count[dev];
 }
 
 template <int D>
@@ -171,18 +183,23 @@ extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_d
   prm.segs = segs_dev;
   prm.work = work_dev;
   prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.n_work = n_work;
   prm.heads = heads;
   prm.scale_log2 = scale * 1.4426950408889634f;
 
+  // Persistent: one CTA per SM (or fewer if there are fewer items).
+  const int sms = sm_count();
+  if (sms <= 0) return MF_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(n_work < sms ? n_work : sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (head_dim == 128) {
     if (!prepare_attention_kernel<128>()) return MF_ERR_CUDA;
     mf::packed_attention_kernel<128>
-        <<<n_work, mf::kAttnThreads, mf::AttnConfig<128>::kSmemBytes, s>>>(tq, tk, tv, prm);
+        <<<grid, mf::kAttnThreads, mf::AttnConfig<128>::kSmemBytes, s>>>(tq, tk, tv, prm);
   } else {
     if (!prepare_attention_kernel<64>()) return MF_ERR_CUDA;
     mf::packed_attention_kernel<64>
-        <<<n_work, mf::kAttnThreads, mf::AttnConfig<64>::kSmemBytes, s>>>(tq, tk, tv, prm);
+        <<<grid, mf::kAttnThreads, mf::AttnConfig<64>::kSmemBytes, s>>>(tq, tk, tv, prm);
   }
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
 }

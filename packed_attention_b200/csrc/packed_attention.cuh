@@ -6,39 +6,52 @@
 //  cumulative offsets. The pages run it with FlashAttention's var-len
 //  kernels; this kernel is its own design for sm_100a.]
 //
-// One CTA computes one work item: 128 query rows of one head of one sample,
-// attending over the sample's L keys in steps of 128.
+// Persistent: one CTA per SM walks the longest-first work list with a
+// stride of gridDim.x. A work item is 256 query rows of one head of one
+// sample, split into two 128-row sub-tiles a and b that share every K/V tile
+// (b is skipped when it starts past the sample end). Keys are visited in
+// steps of 128.
 //
-//   warp 4 (one lane)  TMA producer: the Q tile once, then K_j and V_j tiles
-//                      into a ring of NS shared-memory stages (128-byte
-//                      swizzled boxes of 128 rows x 64 dims).
-//   warp 5 (one lane)  MMA issuer: S_j = Q K_j^T (both operands in shared
-//                      memory, fp32 accumulator in TMEM, two S buffers), and
-//                      O += P_j V_j (P from TMEM, V from shared memory, O in
-//                      TMEM). Completion is signalled with tcgen05.commit.
-//                      Warp 5 also owns the TMEM allocation.
-//   warps 0-3          softmax, one thread per query row: load the S row from
-//                      TMEM, mask keys past the sample end, online max and
-//                      sum in the exp2 domain, write P (bf16) to TMEM, and
-//                      rescale O in TMEM only when the running max grew by
-//                      more than 2^8 (otherwise keep the stale max: p <= 256
-//                      stays exact enough in bf16 and cannot overflow fp32).
-//                      At the end they normalise O by the row sum and store
-//                      bf16 rows, skipping rows past the sample end.
+//   warps 0-3 / 4-7  softmax for sub-tile a / b, one thread per query row:
+//                    load the S row from TMEM, mask keys past the sample
+//                    end, online max and sum in the exp2 domain, write P
+//                    (bf16) back into TMEM over S, and rescale O in TMEM only
+//                    when the running max grew by more than 2^8 (a stale max
+//                    keeps p <= 256: exact enough in bf16, safe in fp32). At
+//                    the end of an item: O / l -> bf16 rows, skipping rows
+//                    past the sample end.
+//   warp 8 (1 lane)  TMA producer: both Q sub-tiles per item, then K_j, V_j
+//                    into a ring of shared-memory stages (128-byte swizzled
+//                    boxes of 128 rows x 64 dims).
+//   warp 9 (1 lane)  MMA issuer (also owns the TMEM allocation):
+//                      S_a(0) S_b(0) | PV_a(j) S_a(j+1) PV_b(j) S_b(j+1) | ...
+//                    S = Q K^T with both operands in shared memory; O += P V
+//                    with P from TMEM and V (an MN-major operand) from shared
+//                    memory; fp32 accumulators in TMEM. While softmax a works
+//                    on S_a(j+1) the tensor core runs PV_b(j) and S_b(j+1),
+//                    and the other way round.
 //
-// TMEM columns (512 allocated): S0 [0,128), S1 [128,256), O [256,256+d),
-// P0 [384,448), P1 [448,512) -- P holds 128 bf16 per row, two per column.
+// TMEM (512 columns): S_a [0,128) O_a [128,256) S_b [256,384) O_b [384,512).
+// P_t(j) overwrites the first 64 columns of S_t after the softmax has read
+// S_t(j); S_t(j+1) is issued after PV_t(j), and tcgen05 MMAs of one thread
+// execute in issue order, so P is read before it is overwritten.
 //
-// Order of tensor-core work: S0, S1, PV0, S2, PV1, S3, ... S_{j+1} is issued
-// before waiting for P_j, so the tensor core computes the next scores while
-// the softmax threads work on the current ones. A commit tracks every earlier
-// tcgen05 operation of the issuing thread, so when S_j's commit fires PV_{j-2}
-// is also complete and the P buffer (j mod 2) may be overwritten.
+// Synchronisation (mbarriers; every arrival is waited for exactly once, in
+// order, so a parity wait can never confuse two phases):
+//   q_full / q_empty   producer <-> MMA, one phase per item
+//   kv_full / kv_empty producer <-> MMA, per ring stage
+//   s_full[t]          MMA -> softmax t, one phase per S_t. A commit tracks
+//                      all earlier MMAs of the thread, so when S_t(j) lands,
+//                      PV_t(j-1) is complete too: O_t may be rescaled and
+//                      P_t may be overwritten without another wait.
+//   p_full[t]          softmax t (4 warps) -> MMA, one phase per P_t
+//   o_ready[t]         MMA -> softmax t after the item's last PV_t
 //
 // Every wait is bounded (kWaitLimitNs). A wait that runs out records
-// MF_ERR_TIMEOUT in the device error word, raises the CTA's abort flag, and
-// every role then leaves its loop, waits (bounded) for its own copies and
-// MMAs in flight, and the TMEM is released before the CTA exits.
+// MF_ERR_TIMEOUT in the device error word and raises the CTA's abort flag;
+// every role leaves its loop, the producer waits (bounded) for its copies
+// in flight, the MMA warp commits and waits for its MMAs, and TMEM is
+// released before the CTA exits.
 #pragma once
 
 #include <cuda.h>
@@ -53,37 +66,70 @@ namespace mf {
 __device__ int32_t g_device_error;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
-constexpr int kAttnThreads = 192;
-constexpr int kBlockM = MF_TILE_M;
-constexpr int kBlockN = MF_TILE_N;
-constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16 (128 bytes, one swizzle span)
+constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms for in-flight work on abort
+constexpr int kAttnThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kSubM = 128;             // rows of one query sub-tile (MMA M)
+constexpr int kBlockN = MF_TILE_N;     // keys per step (MMA N of S, K of PV)
+constexpr int kBoxBytes = 128 * 128;   // 128 rows x 64 bf16 = one 128-byte swizzle span
+constexpr int kMaxStages = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+static_assert(MF_TILE_M == 2 * kSubM, "a work item is two query sub-tiles");
+
+__device__ __forceinline__ uint32_t col_s(int t) { return 256u * static_cast<uint32_t>(t); }
+__device__ __forceinline__ uint32_t col_o(int t) { return 256u * static_cast<uint32_t>(t) + 128u; }
 
 template <int D>
 struct AttnConfig {
   static constexpr int kBoxes = D / 64;
-  static constexpr int kTileBytes = kBlockM * D * 2;
-  static constexpr int kStages = D == 128 ? 3 : 4;
-  static constexpr int kSmemBytes = kTileBytes * (1 + kStages) + 1024;
+  static constexpr int kTileBytes = kSubM * D * 2;  // one 128-row tile of Q, K or V
+  static constexpr int kStages = D == 128 ? 3 : 6;
+  static constexpr int kSmemBytes = kTileBytes * (2 + kStages) + 1024;
+  static_assert(kStages <= kMaxStages, "ring too deep");
 };
 
 struct AttnParams {
   const mf_segment* segs;
   const mf_work_item* work;
   __nv_bfloat16* out;
+  int n_work;
   int heads;
   float scale_log2;  // softmax scale * log2(e)
 };
 
+struct ItemInfo {
+  int seg_start;
+  int seg_len;
+  int head;
+  int q0;      // first query row of sub-tile a
+  int n_kv;    // key steps
+  bool b_valid;
+};
+
+__device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int idx) {
+  const mf_work_item wi = p.work[idx];
+  const mf_segment sg = p.segs[wi.seg];
+  ItemInfo it;
+  it.seg_start = sg.start;
+  it.seg_len = sg.len;
+  it.head = wi.head;
+  it.q0 = sg.start + wi.q_tile * MF_TILE_M;
+  it.n_kv = (sg.len + kBlockN - 1) / kBlockN;
+  it.b_valid = it.q0 + kSubM < sg.start + sg.len;
+  return it;
+}
+
 struct SharedCtl {
   uint64_t q_full;
-  uint64_t kv_full[4];
-  uint64_t kv_empty[4];
+  uint64_t q_empty;
+  uint64_t kv_full[kMaxStages];
+  uint64_t kv_empty[kMaxStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t pv_done;
+  uint64_t o_ready[2];
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort;
@@ -120,15 +166,31 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-// One 128-column TMEM row per thread (32 lanes per warp), waited.
-__device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, float (&v)[128]) {
+// S (tmem) = Q (smem) K^T (smem): M=128, N=128, K=D in steps of 16. Both are
+// K-major with the 128-byte swizzle: a K step of 16 elements is 32 bytes
+// inside a 128-byte row; 64-element column blocks are one box apart.
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, kBlockN, 0, 0);
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    uint32_t r[64];
-    tmem_ld64_sync(taddr + 64 * c, r);
-#pragma unroll
-    for (int i = 0; i < 64; ++i) v[64 * c + i] = __uint_as_float(r[i]);
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * kBoxBytes + (kk % 4) * 32;
+    mma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+           kIdesc, kk > 0 ? 1u : 0u);
   }
+}
+
+// O (tmem) (+)= P (tmem, bf16) V (smem): M=128, N=D, K=128 keys in steps of
+// 16. V is [keys, d] with d contiguous, an MN-major operand: 16 keys are two
+// 8-row swizzle atoms (2 KB); 64-dim blocks are one box apart (LBO).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                         bool accumulate) {
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < kBlockN / 16; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), kIdesc,
+           (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -144,40 +206,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __shared__ SharedCtl ctl;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + kTile;
+  uint8_t* sQ = smem;                // sub-tile a, then sub-tile b
+  uint8_t* sKV = smem + 2 * kTile;   // NS stages
   volatile int32_t* abort_flag = &ctl.abort;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  const mf_work_item wi = p.work[blockIdx.x];
-  const mf_segment seg = p.segs[wi.seg];
-  const int q0 = seg.start + wi.q_tile * kBlockM;
-  const int seg_end = seg.start + seg.len;
-  const int n_kv = (seg.len + kBlockN - 1) / kBlockN;
-
   if (threadIdx.x == 0) {
     mbar_init(&ctl.q_full, 1);
+    mbar_init(&ctl.q_empty, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&ctl.kv_full[s], 1);
       mbar_init(&ctl.kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&ctl.s_full[b], 1);
-      mbar_init(&ctl.p_full[b], 4);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl.s_full[t], 1);
+      mbar_init(&ctl.p_full[t], 4);
+      mbar_init(&ctl.o_ready[t], 1);
     }
-    mbar_init(&ctl.pv_done, 1);
     mbar_init(&ctl.drain, 1);
     ctl.abort = 0;
     fence_mbarrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmap_q);
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&ctl.tmem_base, kTmemCols);
     tmem_relinquish_alloc_permit();
   }
@@ -185,180 +242,216 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = ctl.tmem_base;
+  const int stride = static_cast<int>(gridDim.x);
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------ TMA producer ---
     if (lane == 0) {
-      int issued = 0;
+      int g = 0;  // tile loads issued into the ring so far
+      int k = 0;  // items started
       bool ok = true;
-      mbar_arrive_expect_tx(&ctl.q_full, kTile);
+      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride, ++k) {
+        const ItemInfo it = load_item(p, idx);
+        if (k > 0 && !wait_bar(&ctl.q_empty, (k - 1) & 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl.q_full, 2 * kTile);
 #pragma unroll
-      for (int b = 0; b < Cfg::kBoxes; ++b)
-        tma_load_3d(sQ + b * kBoxBytes, &tmap_q, &ctl.q_full, 64 * b, wi.head, q0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        for (int which = 0; which < 2; ++which) {
-          const int i = 2 * j + which;
-          const int st = i % NS;
-          if (!wait_bar(&ctl.kv_empty[st], ((i / NS) & 1) ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&ctl.kv_full[st], kTile);
-          const CUtensorMap* map = which ? &tmap_v : &tmap_k;
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int b = 0; b < Cfg::kBoxes; ++b)
-            tma_load_3d(sKV + st * kTile + b * kBoxBytes, map, &ctl.kv_full[st], 64 * b, wi.head,
-                        seg.start + j * kBlockN);
-          issued = i + 1;
+            tma_load_3d(sQ + t * kTile + b * kBoxBytes, &tmap_q, &ctl.q_full, 64 * b, it.head,
+                        it.q0 + t * kSubM);
+        for (int j = 0; j < it.n_kv && ok; ++j) {
+          for (int which = 0; which < 2; ++which, ++g) {
+            const int st = g % NS;
+            if (!wait_bar(&ctl.kv_empty[st], ((g / NS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&ctl.kv_full[st], kTile);
+            const CUtensorMap* map = which ? &tmap_v : &tmap_k;
+#pragma unroll
+            for (int b = 0; b < Cfg::kBoxes; ++b)
+              tma_load_3d(sKV + st * kTile + b * kBoxBytes, map, &ctl.kv_full[st], 64 * b, it.head,
+                          it.seg_start + j * kBlockN);
+          }
         }
       }
       if (!ok) {
-        // Let the copies already issued land before the CTA can exit.
-        wait_slow(&ctl.q_full, 0, nullptr, 100000000ull);
-        for (int i = issued - NS > 0 ? issued - NS : 0; i < issued; ++i)
-          wait_slow(&ctl.kv_full[i % NS], (i / NS) & 1, nullptr, 100000000ull);
+        // Let every copy already issued land before the CTA can exit.
+        if (k > 0) wait_slow(&ctl.q_full, (k - 1) & 1, nullptr, kDrainLimitNs);
+        for (int i = g - NS > 0 ? g - NS : 0; i < g; ++i)
+          wait_slow(&ctl.kv_full[i % NS], (i / NS) & 1, nullptr, kDrainLimitNs);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // -------------------------------------------------------- MMA issuer ---
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
-      constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, D, 0, 1);
-      const uint32_t q_addr = smem_addr(sQ);
+      const uint32_t q_addr[2] = {smem_addr(sQ), smem_addr(sQ + kTile)};
       const uint32_t kv_addr = smem_addr(sKV);
-      const int total_loads = 2 * n_kv;
-      bool ok = wait_bar(&ctl.q_full, 0, abort_flag);
-      tc_fence_after_sync();
-
-      // S_jj = Q K_jj^T into S buffer (jj mod 2).
-      auto issue_s = [&](int jj) -> bool {
-        const int i = 2 * jj;
-        const int st = i % NS;
-        if (!wait_bar(&ctl.kv_full[st], (i / NS) & 1, abort_flag)) return false;
+      // Loads this CTA will consume: a stage is released only if it will be
+      // refilled, so that no arrival is left pending when the CTA exits.
+      int total_loads = 0;
+      for (int idx = blockIdx.x; idx < p.n_work; idx += stride) total_loads += 2 * load_item(p, idx).n_kv;
+      int g = 0;        // tile loads consumed so far
+      int k = 0;        // items done
+      uint32_t np[2] = {0, 0};  // P phases consumed per sub-tile
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride, ++k) {
+        const ItemInfo it = load_item(p, idx);
+        const bool has_next = idx + stride < p.n_work;
+        const int n = it.n_kv;
+        const int nt = it.b_valid ? 2 : 1;
+        if (!wait_bar(&ctl.q_full, k & 1, abort_flag)) { ok = false; break; }
         tc_fence_after_sync();
-        const uint32_t k_addr = kv_addr + st * kTile;
-        const uint32_t d_tmem = tmem + ((jj & 1) ? kColS1 : kColS0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kBoxBytes + (kk % 4) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024),
-                 smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+        // S_t(0) for both sub-tiles.
+        {
+          const int st = g % NS;
+          if (!wait_bar(&ctl.kv_full[st], (g / NS) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          for (int t = 0; t < nt; ++t) {
+            issue_qk<D>(tmem + col_s(t), q_addr[t], kv_addr + st * kTile);
+            mma_commit(&ctl.s_full[t]);
+          }
+          if (n == 1 && has_next) mma_commit(&ctl.q_empty);
+          if (g + NS < total_loads) mma_commit(&ctl.kv_empty[st]);
+          ++g;
         }
-        if (i + NS < total_loads) mma_commit(&ctl.kv_empty[st]);
-        mma_commit(&ctl.s_full[jj & 1]);
-        return true;
-      };
-
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv && !issue_s(j + 1)) { ok = false; break; }
-        if (!wait_bar(&ctl.p_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after_sync();
-        const int i = 2 * j + 1;
-        const int st = i % NS;
-        if (!wait_bar(&ctl.kv_full[st], (i / NS) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after_sync();
-        const uint32_t v_addr = kv_addr + st * kTile;
-        const uint32_t p_tmem = tmem + ((j & 1) ? kColP1 : kColP0);
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          // V is [keys, d] with d contiguous: an MN-major B operand. 16 keys per
-          // step = two 8-row swizzle atoms (2 KB); d blocks of 64 are a box apart.
-          mma_ts(tmem + kColO, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024),
-                 kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int j = 0; j < n && ok; ++j) {
+          const int gv = g;      // V_j
+          const int gk = g + 1;  // K_{j+1}
+          const bool more = j + 1 < n;
+          const int sv = gv % NS, sk = gk % NS;
+          if (!wait_bar(&ctl.kv_full[sv], (gv / NS) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          if (more) {
+            if (!wait_bar(&ctl.kv_full[sk], (gk / NS) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after_sync();
+          }
+          for (int t = 0; t < nt; ++t) {
+            if (!wait_bar(&ctl.p_full[t], np[t] & 1, abort_flag)) { ok = false; break; }
+            ++np[t];
+            tc_fence_after_sync();
+            issue_pv<D>(tmem + col_o(t), tmem + col_s(t), kv_addr + sv * kTile, j > 0);
+            if (!more) mma_commit(&ctl.o_ready[t]);
+            if (more) {
+              issue_qk<D>(tmem + col_s(t), q_addr[t], kv_addr + sk * kTile);
+              mma_commit(&ctl.s_full[t]);
+            }
+          }
+          if (!ok) break;
+          if (gv + NS < total_loads) mma_commit(&ctl.kv_empty[sv]);
+          g = gv + 1;
+          if (more) {
+            if (j + 1 == n - 1 && has_next) mma_commit(&ctl.q_empty);
+            if (gk + NS < total_loads) mma_commit(&ctl.kv_empty[sk]);
+            g = gk + 1;
+          }
         }
-        if (i + NS < total_loads) mma_commit(&ctl.kv_empty[st]);
-        mma_commit(&ctl.pv_done);
       }
       if (!ok) {
         // Every MMA issued so far must finish before TMEM is released.
         mma_commit(&ctl.drain);
-        wait_slow(&ctl.drain, 0, nullptr, 100000000ull);
+        wait_slow(&ctl.drain, 0, nullptr, kDrainLimitNs);
       }
     }
   } else {
     // ----------------------------------------------------------- softmax ---
-    const int row = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int t = warp / 4;  // sub-tile
+    const int wl = warp % 4;
+    const int row = wl * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_off + col_s(t);
+    const uint32_t o_tmem = tmem + lane_off + col_o(t);
     const float sl2 = p.scale_log2;
-    float m = -INFINITY;  // running max of s * scale * log2(e)
-    float l = 0.0f;       // running sum of p
+    const uint64_t sl2x2 = f32x2(sl2, sl2);
+    uint32_t ns = 0;  // S phases consumed
+    uint32_t no = 0;  // O phases consumed
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!warp_wait_bar(&ctl.s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after_sync();
-      float s[128];
-      tmem_ld128_wait(tmem + lane_off + ((j & 1) ? kColS1 : kColS0), s);
-      const int valid = seg.len - j * kBlockN;  // keys of this step inside the sample
-      if (valid < kBlockN) {
+    for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+      const ItemInfo it = load_item(p, idx);
+      if (t == 1 && !it.b_valid) continue;
+      float m = -INFINITY;  // running max of s * scale * log2(e)
+      float l = 0.0f;       // running sum of p
+      for (int j = 0; j < it.n_kv; ++j) {
+        if (!warp_wait_bar(&ctl.s_full[t], ns & 1, abort_flag)) { ok = false; break; }
+        ++ns;
+        tc_fence_after_sync();
+        float s[128];
+        {
+          uint32_t sr[128];
+          tmem_ld128_sync(s_tmem, sr);
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= valid) s[c] = -INFINITY;
-      }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-      const float m_new = fmaxf(m, m_tile);
-      // pv_done must be observed once per phase, in order (a parity wait cannot
-      // tell phase j-1 from phase j-3): PV_{j-1} is waited for here when O has
-      // to be rescaled, otherwise just before P_j is handed to the MMA warp.
-      bool pv_prev_seen = (j == 0);
-      if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
-        const float factor = ex2_approx(m - m_new);  // 0 on the first step
-        l *= factor;
-        if (j > 0) {
-          // O holds PV_0..PV_{j-1}: wait for the last one, then scale the row.
-          if (!warp_wait_bar(&ctl.pv_done, (j - 1) & 1, abort_flag)) { ok = false; break; }
-          pv_prev_seen = true;
-          tc_fence_after_sync();
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            const uint32_t ta = tmem + lane_off + kColO + 32 * c;
-            tmem_ld32_sync(ta, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
-            tmem_st32_sync(ta, r);
-          }
+          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
         }
-        m = m_new;
-      }
-      float l0 = 0.f, l1 = 0.f;
-      uint32_t pk[64];
+        const int valid = it.seg_len - j * kBlockN;  // keys of this step inside the sample
+        if (valid < kBlockN) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, -m));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, -m));
-        l0 += p0;
-        l1 += p1;
-        pk[c] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < 128; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
+        float mx2 = fmax3(s[6], s[7], s[8]), mx3 = fmax3(s[9], s[10], s[11]);
+#pragma unroll
+        for (int c = 12; c < 124; c += 8) {
+          mx0 = fmax3(mx0, s[c], s[c + 1]);
+          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+        }
+        mx0 = fmax3(mx0, s[124], s[125]);
+        mx1 = fmax3(mx1, s[126], s[127]);
+        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        const float m_new = fmaxf(m, m_tile);
+        if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
+          // S_t(j) has landed, so PV_t(j-1) is complete: O_t may be rescaled.
+          const float factor = ex2_approx(m - m_new);  // 0 on the first step
+          l *= factor;
+          if (j > 0) {
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32_sync(o_tmem + 32 * c, r);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
+              tmem_st32_sync(o_tmem + 32 * c, r);
+            }
+          }
+          m = m_new;
+        }
+        const uint64_t neg_m = f32x2(-m, -m);
+        uint64_t acc0 = f32x2(0.f, 0.f), acc1 = acc0;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const uint64_t x = fma_f32x2(f32x2(s[2 * c], s[2 * c + 1]), sl2x2, neg_m);
+          float x0, x1;
+          f32x2_split(x, x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (c & 1) acc1 = add_f32x2(acc1, f32x2(p0, p1));
+          else acc0 = add_f32x2(acc0, f32x2(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        float a0, a1, a2, a3;
+        f32x2_split(acc0, a0, a1);
+        f32x2_split(acc1, a2, a3);
+        l += (a0 + a1) + (a2 + a3);
+        tmem_st64_sync(s_tmem, pk);  // P over the first 64 columns of S
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.p_full[t]);
       }
-      l += l0 + l1;
-      tmem_st64_sync(tmem + lane_off + ((j & 1) ? kColP1 : kColP0), pk);
-      if (!pv_prev_seen && !warp_wait_bar(&ctl.pv_done, (j - 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.p_full[j & 1]);
-    }
-    if (ok && warp_wait_bar(&ctl.pv_done, (n_kv - 1) & 1, abort_flag)) {
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 rows of this sub-tile ----
+      if (!warp_wait_bar(&ctl.o_ready[t], no & 1, abort_flag)) { ok = false; break; }
+      ++no;
       tc_fence_after_sync();
-      const int q_row = q0 + row;
+      const int q_row = it.q0 + t * kSubM + row;
+      const bool store = q_row < it.seg_start + it.seg_len;
       const float inv_l = 1.0f / l;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(q_row) * p.heads + wi.head) * D);
+      uint4* dst = reinterpret_cast<uint4*>(p.out) +
+                   (static_cast<size_t>(q_row) * p.heads + it.head) * (D / 8);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32_sync(tmem + lane_off + kColO + 32 * c, r);
-        if (q_row < seg_end) {
+        tmem_ld32_sync(o_tmem + 32 * c, r);
+        if (store) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 o;
@@ -376,7 +469,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // ---------------------------------------------------------- teardown ---
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);

@@ -6,7 +6,7 @@
 //  packed with their text under a fixed token budget; attention uses
 //  per-sample cumulative offsets. Video overview, 00:04:03: no padding.]
 //
-// The work list holds one item per (sample, head, 128-row query tile). Items
+// The work list holds one item per (sample, head, 256-row query tile). Items
 // are ordered by sample length, longest first, because an item's cost grows
 // with the number of keys it attends over (its sample's length): handing the
 // longest items out first keeps the last wave of the persistent kernel short.
