@@ -215,6 +215,16 @@ mf_status mf_joint_attn_fwd_static_scratch(
     void* out, void* stream);
 
 /*
+ * mf_selftest_exp2 -- diagnostic: y[i] = 2^x[i] computed by the attention
+ * softmax's FMA-pipe exponential (the share of exponentials it keeps off the
+ * MUFU unit), so its accuracy can be checked on its own. x, y: device fp32
+ * arrays of n elements (n >= 0; n odd is fine). Inputs below -125 give
+ * 2^-125-scale values (zero to bf16), -inf included. Asynchronous on
+ * `stream`; MF_ERR_INVALID_ARG for NULL pointers or n < 0.
+ */
+mf_status mf_selftest_exp2(const float* x, float* y, int32_t n, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the error the kernels
  * recorded on the current device since the last call (MF_OK if none,
  * MF_ERR_TIMEOUT if a pipeline wait ran out of time and the kernel gave up).

@@ -97,7 +97,13 @@ bool prepare_attention_kernel() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   std::call_once(once[dev], [dev] {
-    ok[dev] = cudaFuncSetAttribute(mf::packed_attention_kernel<D>,
+    // The kernel re-splits its registers between warpgroups; that only works
+    // if it is launched with at least kMinLaunchRegs per thread (otherwise the
+    // softmax warpgroups would wait forever for registers): refuse instead.
+    cudaFuncAttributes attr;
+    ok[dev] = cudaFuncGetAttributes(&attr, mf::packed_attention_kernel<D>) == cudaSuccess &&
+              attr.numRegs >= mf::kMinLaunchRegs &&
+              cudaFuncSetAttribute(mf::packed_attention_kernel<D>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    mf::AttnConfig<D>::kSmemBytes) == cudaSuccess;
   });
@@ -225,6 +231,28 @@ extern "C" mf_status mf_joint_attn_fwd(const void* q, const void* k, const void*
   if (st != MF_OK) return st;
   return mf_packed_attention(v, segs_dev, n_samples, work_dev, n_work, total_tokens, heads,
                              head_dim, softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+namespace {
+
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.0f;
+  float y0, y1;
+  mf::exp2_fma_x2(x0, x1, y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+
+}  // namespace
+
+extern "C" mf_status mf_selftest_exp2(const float* x, float* y, int32_t n, void* stream) {
+  if (!x || !y || n < 0) return MF_ERR_INVALID_ARG;
+  if (n == 0) return MF_OK;
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
 }
 
 extern "C" mf_status mf_get_device_error(void* stream) {

@@ -23,6 +23,9 @@
 //   warp 8 (1 lane)  TMA producer: both Q sub-tiles per item, then K_j, V_j
 //                    into a ring of shared-memory stages (128-byte swizzled
 //                    boxes of 128 rows x 64 dims).
+//   warps 10-11      idle; they complete warpgroup 2 so that its registers
+//                    can be handed to the softmax warpgroups (setmaxnreg:
+//                    softmax 200 per thread, warpgroup 2 96 per thread).
 //   warp 9 (1 lane)  MMA issuer (also owns the TMEM allocation):
 //                      S_a(0) S_b(0) | PV_a(j) S_a(j+1) PV_b(j) S_b(j+1) | ...
 //                    S = Q K^T with both operands in shared memory; O += P V
@@ -44,7 +47,9 @@
 //                      all earlier MMAs of the thread, so when S_t(j) lands,
 //                      PV_t(j-1) is complete too: O_t may be rescaled and
 //                      P_t may be overwritten without another wait.
-//   p_full[t]          softmax t (4 warps) -> MMA, one phase per P_t
+//   p_half[t][h]       softmax t (4 warps) -> MMA, one phase per half (64
+//                      keys) of P_t: the first half of PV_t starts while the
+//                      softmax computes the second half's exponentials
 //   o_ready[t]         MMA -> softmax t after the item's last PV_t
 //
 // Every wait is bounded (kWaitLimitNs). A wait that runs out records
@@ -67,7 +72,13 @@ __device__ int32_t g_device_error;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms for in-flight work on abort
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;
+constexpr uint32_t kSoftmaxRegs = 200;   // per thread, warpgroups 0 and 1
+constexpr uint32_t kControlRegs = 96;    // per thread, warpgroup 2
+// The split must fit in what the CTA is launched with (384 x regs/thread):
+// the host refuses to launch if the compiled kernel uses fewer registers.
+constexpr int kMinLaunchRegs = (2 * 128 * kSoftmaxRegs + 128 * kControlRegs + kAttnThreads - 1) /
+                               kAttnThreads;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kSubM = 128;             // rows of one query sub-tile (MMA M)
@@ -76,6 +87,8 @@ constexpr int kBoxBytes = 128 * 128;   // 128 rows x 64 bf16 = one 128-byte swiz
 constexpr int kMaxStages = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// One column pair in kPolyEvery takes its exponentials on the FMA pipe (0: none).
+constexpr int kPolyEvery = 0;
 
 static_assert(MF_TILE_M == 2 * kSubM, "a work item is two query sub-tiles");
 
@@ -86,7 +99,8 @@ template <int D>
 struct AttnConfig {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kSubM * D * 2;  // one 128-row tile of Q, K or V
-  static constexpr int kStages = D == 128 ? 3 : 6;
+  // Deep enough that each K/V load is requested a full key step before use.
+  static constexpr int kStages = D == 128 ? 4 : 6;
   static constexpr int kSmemBytes = kTileBytes * (2 + kStages) + 1024;
   static_assert(kStages <= kMaxStages, "ring too deep");
 };
@@ -128,14 +142,16 @@ struct SharedCtl {
   uint64_t kv_full[kMaxStages];
   uint64_t kv_empty[kMaxStages];
   uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t p_half[2][2];  // first / second 64 keys of P_t
   uint64_t o_ready[2];
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort;
 };
 
-__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile int32_t* abort_flag,
+// Inlined: a call inside a setmaxnreg region would have to fit the caller's
+// register budget at every call site, which ptxas cannot arrange.
+__device__ __forceinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile int32_t* abort_flag,
                                        uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
@@ -166,30 +182,61 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// 2^x for two lanes on the FMA pipe, to take a share of the exponentials off
+// the MUFU unit (whose 16 results per clock per SM equal the tensor core's
+// score rate). Cody-Waite reduction x = n + f, n = rint(x), f in [-1/2, 1/2]
+// (rint by adding 1.5 * 2^23), 2^f by a cubic with minimax relative error
+// 7.5e-5 (coefficients from fit_exp2_poly.py), and 2^n added to the exponent
+// field with one integer multiply-add. x is clamped at -125 so that n + the
+// exponent of 2^f stays a normal exponent (2^-125 ~ 2.4e-38 is zero to bf16).
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f32x2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t xr = add_f32x2(x, f32x2(kRound, kRound));        // n in the low mantissa bits
+  const uint64_t n = add_f32x2(xr, f32x2(-kRound, -kRound));      // rint(x)
+  const uint64_t f = fma_f32x2(n, f32x2(-1.0f, -1.0f), x);        // x - n, exact
+  uint64_t q = fma_f32x2(f32x2(kC3, kC3), f, f32x2(kC2, kC2));
+  q = fma_f32x2(q, f, f32x2(kC1, kC1));
+  q = fma_f32x2(q, f, f32x2(kC0, kC0));
+  float q0, q1, r0, r1;
+  f32x2_split(q, q0, q1);
+  f32x2_split(xr, r0, r1);
+  y0 = __uint_as_float(imad(__float_as_uint(r0), 1u << 23, __float_as_uint(q0)));
+  y1 = __uint_as_float(imad(__float_as_uint(r1), 1u << 23, __float_as_uint(q1)));
+}
+
+// Shared-memory descriptors are built once; a descriptor for base + off is
+// the base descriptor plus off >> 4 (the start-address field is the low 14
+// bits, and shared addresses stay below 256 KB, so the add never carries out
+// of it). Building them per MMA would cost a dependent integer chain of ~100
+// cycles on the issuing thread, longer than the 64-cycle MMA itself.
+
 // S (tmem) = Q (smem) K^T (smem): M=128, N=128, K=D in steps of 16. Both are
 // K-major with the 128-byte swizzle: a K step of 16 elements is 32 bytes
 // inside a 128-byte row; 64-element column blocks are one box apart.
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
   constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, kBlockN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * kBoxBytes + (kk % 4) * 32;
-    mma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-           kIdesc, kk > 0 ? 1u : 0u);
+    const uint64_t off = static_cast<uint64_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4);
+    mma_ss(d_tmem, q_desc + off, k_desc + off, kIdesc, kk > 0 ? 1u : 0u);
   }
 }
 
-// O (tmem) (+)= P (tmem, bf16) V (smem): M=128, N=D, K=128 keys in steps of
-// 16. V is [keys, d] with d contiguous, an MN-major operand: 16 keys are two
-// 8-row swizzle atoms (2 KB); 64-dim blocks are one box apart (LBO).
-template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
+// O (tmem) (+)= P (tmem, bf16) V (smem) over keys [16*k0, 16*k1): M=128, N=D,
+// K=16 per MMA. V is [keys, d] with d contiguous, an MN-major operand: 16
+// keys are two 8-row swizzle atoms (2 KB); 64-dim blocks are one box apart
+// (the descriptor's leading byte offset).
+template <int D, int k0, int k1>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc,
                                          bool accumulate) {
   constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, D, 0, 1);
 #pragma unroll
-  for (int kk = 0; kk < kBlockN / 16; ++kk)
-    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), kIdesc,
+  for (int kk = k0; kk < k1; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, v_desc + static_cast<uint64_t>(kk * (2048 >> 4)), kIdesc,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -222,7 +269,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&ctl.s_full[t], 1);
-      mbar_init(&ctl.p_full[t], 4);
+      mbar_init(&ctl.p_half[t][0], 4);
+      mbar_init(&ctl.p_half[t][1], 4);
       mbar_init(&ctl.o_ready[t], 1);
     }
     mbar_init(&ctl.drain, 1);
@@ -243,7 +291,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = ctl.tmem_base;
   const int stride = static_cast<int>(gridDim.x);
-
+  if (warp >= 8) {
+    // Warpgroup 2 (producer, MMA issuer, two idle warps) gives registers away.
+    setmaxnreg_dec<kControlRegs>();
+  }
   if (warp == kProducerWarp) {
     // ------------------------------------------------------ TMA producer ---
     if (lane == 0) {
@@ -283,8 +334,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------- MMA issuer ---
     if (lane == 0) {
-      const uint32_t q_addr[2] = {smem_addr(sQ), smem_addr(sQ + kTile)};
-      const uint32_t kv_addr = smem_addr(sKV);
+      const uint64_t q_desc[2] = {smem_desc_sw128(smem_addr(sQ), 16, 1024),
+                                  smem_desc_sw128(smem_addr(sQ + kTile), 16, 1024)};
+      // K stages as K-major operands, V stages as MN-major operands.
+      const uint64_t k_desc0 = smem_desc_sw128(smem_addr(sKV), 16, 1024);
+      const uint64_t v_desc0 = smem_desc_sw128(smem_addr(sKV), kBoxBytes, 1024);
+      constexpr uint64_t kStageStep = static_cast<uint64_t>(kTile >> 4);
       // Loads this CTA will consume: a stage is released only if it will be
       // refilled, so that no arrival is left pending when the CTA exits.
       int total_loads = 0;
@@ -306,7 +361,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!wait_bar(&ctl.kv_full[st], (g / NS) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
           for (int t = 0; t < nt; ++t) {
-            issue_qk<D>(tmem + col_s(t), q_addr[t], kv_addr + st * kTile);
+            issue_qk<D>(tmem + col_s(t), q_desc[t], k_desc0 + st * kStageStep);
             mma_commit(&ctl.s_full[t]);
           }
           if (n == 1 && has_next) mma_commit(&ctl.q_empty);
@@ -320,18 +375,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int sv = gv % NS, sk = gk % NS;
           if (!wait_bar(&ctl.kv_full[sv], (gv / NS) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          if (more) {
-            if (!wait_bar(&ctl.kv_full[sk], (gk / NS) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after_sync();
-          }
           for (int t = 0; t < nt; ++t) {
-            if (!wait_bar(&ctl.p_full[t], np[t] & 1, abort_flag)) { ok = false; break; }
+            // PV in two halves: the first 64 keys start while the softmax is
+            // still computing the exponentials of the second 64.
+            if (!wait_bar(&ctl.p_half[t][0], np[t] & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after_sync();
+            issue_pv<D, 0, 4>(tmem + col_o(t), tmem + col_s(t), v_desc0 + sv * kStageStep, j > 0);
+            if (!wait_bar(&ctl.p_half[t][1], np[t] & 1, abort_flag)) { ok = false; break; }
             ++np[t];
             tc_fence_after_sync();
-            issue_pv<D>(tmem + col_o(t), tmem + col_s(t), kv_addr + sv * kTile, j > 0);
+            issue_pv<D, 4, 8>(tmem + col_o(t), tmem + col_s(t), v_desc0 + sv * kStageStep, true);
             if (!more) mma_commit(&ctl.o_ready[t]);
             if (more) {
-              issue_qk<D>(tmem + col_s(t), q_addr[t], kv_addr + sk * kTile);
+              if (t == 0) {
+                // K_{j+1} is needed only now, after PV_a(j) has been queued.
+                if (!wait_bar(&ctl.kv_full[sk], (gk / NS) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after_sync();
+              }
+              issue_qk<D>(tmem + col_s(t), q_desc[t], k_desc0 + sk * kStageStep);
               mma_commit(&ctl.s_full[t]);
             }
           }
@@ -351,8 +412,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         wait_slow(&ctl.drain, 0, nullptr, kDrainLimitNs);
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ----------------------------------------------------------- softmax ---
+    setmaxnreg_inc<kSoftmaxRegs>();
     const int t = warp / 4;  // sub-tile
     const int wl = warp % 4;
     const int row = wl * 32 + lane;
@@ -417,25 +479,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         const uint64_t neg_m = f32x2(-m, -m);
         uint64_t acc0 = f32x2(0.f, 0.f), acc1 = acc0;
-        uint32_t pk[64];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const uint64_t x = fma_f32x2(f32x2(s[2 * c], s[2 * c + 1]), sl2x2, neg_m);
-          float x0, x1;
-          f32x2_split(x, x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          if (c & 1) acc1 = add_f32x2(acc1, f32x2(p0, p1));
-          else acc0 = add_f32x2(acc0, f32x2(p0, p1));
-          pk[c] = pack_bf16x2(p0, p1);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int e = 64 * h + 2 * c;
+            const uint64_t x = fma_f32x2(f32x2(s[e], s[e + 1]), sl2x2, neg_m);
+            float x0, x1, p0, p1;
+            f32x2_split(x, x0, x1);
+            if (kPolyEvery > 0 && c % kPolyEvery == kPolyEvery - 1) {
+              exp2_fma_x2(x0, x1, p0, p1);  // a share of the exponentials on the FMA pipe
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            if (c & 1) acc1 = add_f32x2(acc1, f32x2(p0, p1));
+            else acc0 = add_f32x2(acc0, f32x2(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          // P over the first 64 columns of S, 32 columns (64 keys) at a time.
+          tmem_st32_sync(s_tmem + 32 * h, pk);
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.p_half[t][h]);
         }
         float a0, a1, a2, a3;
         f32x2_split(acc0, a0, a1);
         f32x2_split(acc1, a2, a3);
         l += (a0 + a1) + (a2 + a3);
-        tmem_st64_sync(s_tmem, pk);  // P over the first 64 columns of S
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl.p_full[t]);
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 rows of this sub-tile ----

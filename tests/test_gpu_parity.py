@@ -203,3 +203,28 @@ def test_explicit_softmax_scale(cuda_device):
         ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, scale=scale)
         max_abs, rel_rms = errors(bf16_to_f64(out), ref)
         assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (scale, max_abs, rel_rms)
+
+
+def test_fma_pipe_exp2_accuracy(cuda_device):
+    """The softmax's polynomial exp2 (Cody-Waite reduction + minimax cubic)
+    against fp64: relative error below 1e-4 wherever the result is normal."""
+    import ctypes
+    from packed_attention_b200 import _native
+    xs = np.concatenate([np.linspace(-125.0, 8.0, 1_000_001), np.arange(-125, 9, dtype=np.float64),
+                         np.arange(-125, 9) + 0.5, [0.0, -0.0, 7.999999, -1e-7, 1e-7]])
+    x = torch.tensor(xs, dtype=torch.float32, device=cuda_device)
+    y = torch.empty_like(x)
+    st = torch.cuda.current_stream()
+    assert _native.lib().mf_selftest_exp2(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()),
+                                          x.numel(), ctypes.c_void_p(st.cuda_stream)) == 0
+    got = y.cpu().numpy().astype(np.float64)
+    ref = np.exp2(x.cpu().numpy().astype(np.float64))
+    rel = np.abs(got / ref - 1.0)
+    assert rel.max() < 1e-4, rel.max()
+    # below the clamp, and for -inf, the result is a tiny positive normal number
+    x2 = torch.tensor([-126.0, -200.0, -float("inf"), -3e38], dtype=torch.float32, device=cuda_device)
+    y2 = torch.empty_like(x2)
+    assert _native.lib().mf_selftest_exp2(ctypes.c_void_p(x2.data_ptr()), ctypes.c_void_p(y2.data_ptr()),
+                                          4, ctypes.c_void_p(st.cuda_stream)) == 0
+    v = y2.cpu().numpy()
+    assert np.all(v > 0) and np.all(v < 3e-38) and np.all(np.isfinite(v))
