@@ -30,6 +30,20 @@ sys.path.insert(0, ROOT)
 
 METRIC = "packed joint-attention TFLOP/s and tokens/s on 1 B200; % of dense-BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCE = os.path.join(ROOT, "packed_attention_b200", "csrc", "packed_attention.cuh")
+# DRAM bytes (read + write) of one attention launch, from one ncu capture of
+# the full workload (profiles/traffic_packed_attention_kernel_*.md), keyed by
+# the kernel source it was taken on: any other source reports null.
+MEASURED_TRAFFIC = {
+    ("3ff3c321b9d5f65e", "hires_2048sq_4to1"): 393_875_712 + 109_401_600,
+}
+
+
+def kernel_traffic(workload_name):
+    import hashlib
+    with open(KERNEL_SOURCE, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    return MEASURED_TRAFFIC.get((sha, workload_name))
 
 
 def parse_args():
@@ -43,6 +57,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="CPU time the reference arm spends over all its steps")
     return ap.parse_args()
 
 
@@ -108,19 +124,22 @@ class ClockSampler:
 
 def oracle_sample_rows(w, rng, n_blocks, block=64):
     """Rows for a bounded oracle sample: blocks of `block` consecutive tokens of
-    one head, drawn in proportion to the tokens of each sample."""
+    one head, drawn in proportion to the tokens of each sample. Returns the
+    distinct flat rows (token * H + head) and their algorithmic FLOPs
+    (4 * d * L of the row's sample each)."""
     lens = np.array(w.seg_lens)
     starts = np.concatenate([[0], np.cumsum(lens)])
+    seg_of_token = np.repeat(np.arange(len(lens)), lens)
     rows = []
-    flops = 0
     for _ in range(n_blocks):
         s = int(rng.choice(len(lens), p=lens / lens.sum()))
         h = int(rng.integers(0, w.heads))
         b = int(rng.integers(0, max(1, lens[s] - block + 1)))
         toks = np.arange(starts[s] + b, starts[s] + min(b + block, lens[s]))
         rows.append(toks * w.heads + h)
-        flops += 4 * w.head_dim * int(lens[s]) * len(toks)
-    return np.unique(np.concatenate(rows)), flops
+    rows = np.unique(np.concatenate(rows))
+    flops = int(4 * w.head_dim * lens[seg_of_token[rows // w.heads]].sum())
+    return rows, flops
 
 
 def oracle_throughput(w, inp, seconds, seed=0):
@@ -141,6 +160,23 @@ def oracle_throughput(w, inp, seconds, seed=0):
         f"query rows in 64-token blocks, {flops / 1e9:.1f} GFLOP, {dt:.1f} s"
 
 
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of per-rank timings (a list of floats) over all ranks."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_throughput(flops_per_replica, tokens_per_replica, world, steps, max_total_ms):
+    """Replicas: every rank runs the whole workload; the job's throughput is all
+    ranks' work divided by the slowest rank's time."""
+    step_s = max_total_ms / steps / 1e3
+    return flops_per_replica * world / step_s / 1e12, tokens_per_replica * world / step_s
+
+
 def run_reference(args, w):
     """Reference arm: the fp64 oracle on host cores, one bounded sample per step."""
     from packed_attention_b200.workloads import make_inputs
@@ -151,13 +187,14 @@ def run_reference(args, w):
     cores = os.cpu_count() or 1
     import oracle
     rng = np.random.default_rng(1234)
-    budget = 150.0 / max(1, args.steps + args.warmup)  # seconds of CPU work per step
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)  # CPU seconds per step
     # calibrate block count per step
     rows, _ = oracle_sample_rows(w, rng, cores)
     t0 = time.perf_counter()
     oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
     per_block = (time.perf_counter() - t0) / cores
     n_blocks = max(1, int(budget / max(per_block, 1e-4)))
+    n_blocks = min(n_blocks, 4 * (w.total_tokens * w.heads) // 64 + 1)  # enough to cover every row
     for _ in range(args.warmup):
         rows, _ = oracle_sample_rows(w, rng, n_blocks)
         oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
@@ -259,10 +296,7 @@ def main():
     total_ms = start.elapsed_time(end)
     pro_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
     att_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
-    timing = torch.tensor([total_ms, pro_ms, att_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(timing, op=dist.ReduceOp.MAX)
-    total_ms, pro_ms, att_ms = timing.tolist()
+    total_ms, pro_ms, att_ms = max_over_ranks([total_ms, pro_ms, att_ms], world, dev)
 
     # ---- end to end through the public API on host buffers (copies timed) ----
     host = {n: t[n].cpu().pin_memory() for n in ("q", "k", "v", *pa.GAMMA_NAMES)}
@@ -282,10 +316,7 @@ def main():
     e_e.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = torch.tensor([e_s.elapsed_time(e_e) / args.e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks([e_s.elapsed_time(e_e) / args.e2e_steps], world, dev)[0]
 
     if world > 1:
         dist.destroy_process_group()
@@ -294,9 +325,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     flops = w.flops
-    step_s = total_ms / K / 1e3
-    value = flops * world / step_s / 1e12
-    tokens_per_s = T * world / step_s
+    value, tokens_per_s = whole_job_throughput(flops, T, world, K, total_ms)
     att_tflops = flops / (att_ms / 1e3) / 1e12
     peak_sus = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     peak_burst = float(peaks["bf16_tflops"])
@@ -328,7 +357,7 @@ def main():
             "kernel": "packed_attention_kernel", "bound": "tensor", "achieved": att_tflops,
             "peak": peak_sus, "unit": "TFLOP/s", "frac": att_tflops / peak_sus,
             "peak_kind": f"{peak_src} bf16 dense, sustained",
-            "frac_of_burst_peak": att_tflops / peak_burst, "traffic": None,
+            "frac_of_burst_peak": att_tflops / peak_burst, "traffic": kernel_traffic(w.name),
             "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_ms,
         },
         "prologue": {

@@ -225,6 +225,17 @@ mf_status mf_joint_attn_fwd_static_scratch(
 mf_status mf_selftest_exp2(const float* x, float* y, int32_t n, void* stream);
 
 /*
+ * mf_selftest_timeout -- diagnostic for the failure path: launches one CTA
+ * whose thread 0 waits, through the same bounded wait the attention kernel
+ * uses, on an mbarrier that nothing ever arrives on. After limit_ns
+ * nanoseconds (1 <= limit_ns <= 10^9) the wait gives up, records
+ * MF_ERR_TIMEOUT in the device error word and the kernel returns normally:
+ * no trap, no fault, the context stays usable. mf_get_device_error() then
+ * reports MF_ERR_TIMEOUT. MF_ERR_INVALID_ARG for a limit out of range.
+ */
+mf_status mf_selftest_timeout(int64_t limit_ns, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the error the kernels
  * recorded on the current device since the last call (MF_OK if none,
  * MF_ERR_TIMEOUT if a pipeline wait ran out of time and the kernel gave up).

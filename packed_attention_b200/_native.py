@@ -62,6 +62,7 @@ SIGNATURES = {
     "mf_joint_attn_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32,
                                                I32, F32, F32, P, P]),
     "mf_selftest_exp2": (I32, [P, P, I32, P]),
+    "mf_selftest_timeout": (I32, [I64, P]),
     "mf_get_device_error": (I32, [P]),
 }
 

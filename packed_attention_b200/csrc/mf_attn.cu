@@ -255,6 +255,28 @@ extern "C" mf_status mf_selftest_exp2(const float* x, float* y, int32_t n, void*
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
 }
 
+namespace {
+
+// One thread waits on an mbarrier that expects one arrival which never comes.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int32_t abort_flag;
+  if (threadIdx.x != 0) return;
+  mf::mbar_init(&bar, 1);
+  abort_flag = 0;
+  mf::fence_mbarrier_init();
+  mf::wait_slow(&bar, 0, &abort_flag, limit_ns);  // records MF_ERR_TIMEOUT when it gives up
+}
+
+}  // namespace
+
+extern "C" mf_status mf_selftest_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000) return MF_ERR_INVALID_ARG;
+  selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_ns));
+  return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
+}
+
 extern "C" mf_status mf_get_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MF_ERR_CUDA;
   int32_t v = 0;

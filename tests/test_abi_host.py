@@ -155,3 +155,10 @@ def test_forward_argument_checks(lib):
     assert _fwd(lib, scale=float("inf")) == -1
     assert _fwd(lib, out=0x10000) == -1        # out aliases q
     assert _fwd(lib, ws=0x10000 - 0x100) == -1  # workspace overlaps q
+
+
+def test_diagnostic_entry_points_reject_bad_arguments(lib):
+    assert lib.mf_selftest_timeout(0, None) == -1
+    assert lib.mf_selftest_timeout(2_000_000_000, None) == -1
+    assert lib.mf_selftest_exp2(None, None, 4, None) == -1
+    assert lib.mf_selftest_exp2(ctypes.c_void_p(16), ctypes.c_void_p(32), -1, None) == -1
