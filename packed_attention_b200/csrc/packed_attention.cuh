@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m = m_new;
         }
         const uint64_t neg_m = f32x2(-m, -m);
-        uint64_t acc0 = f32x2(0.f, 0.f), acc1 = acc0;
+        float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
@@ -494,8 +494,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               p0 = ex2_approx(x0);
               p1 = ex2_approx(x1);
             }
-            if (c & 1) acc1 = add_f32x2(acc1, f32x2(p0, p1));
-            else acc0 = add_f32x2(acc0, f32x2(p0, p1));
+            // Row sum in four scalar chains (packing p0, p1 for a paired add
+            // would cost register moves).
+            if (c & 1) { la1 += p0; lb1 += p1; } else { la0 += p0; lb0 += p1; }
             pk[c] = pack_bf16x2(p0, p1);
           }
           // P over the first 64 columns of S, 32 columns (64 keys) at a time.
@@ -504,10 +505,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl.p_half[t][h]);
         }
-        float a0, a1, a2, a3;
-        f32x2_split(acc0, a0, a1);
-        f32x2_split(acc1, a2, a3);
-        l += (a0 + a1) + (a2 + a3);
+        l += (la0 + la1) + (lb0 + lb1);
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 rows of this sub-tile ----
