@@ -35,7 +35,7 @@ KERNEL_SOURCE = os.path.join(ROOT, "packed_attention_b200", "csrc", "packed_atte
 # the full workload (profiles/traffic_packed_attention_kernel_*.md), keyed by
 # the kernel source it was taken on: any other source reports null.
 MEASURED_TRAFFIC = {
-    ("3ff3c321b9d5f65e", "hires_2048sq_4to1"): 393_875_712 + 109_401_600,
+    ("faf40727676a6f43", "hires_2048sq_4to1"): 397_379_328 + 109_314_304,
 }
 
 
@@ -51,7 +51,9 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--config", default="4",
+                    help="workload index 0-4 (default 4), or 'all' for one report line per "
+                         "workload (timing only, no e2e / CPU baseline)")
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -222,10 +224,59 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def report_all(args):
+    """One JSON line per workload: device time of both stages, TFLOP/s, tokens/s,
+    fraction of the measured peaks (single GPU)."""
+    import torch
+    import packed_attention_b200 as pa
+    from packed_attention_b200.workloads import WORKLOADS, make_inputs
+    peaks, peak_src = load_peaks()
+    dev = torch.device("cuda", 0)
+    for cfg, w in WORKLOADS.items():
+        inp = make_inputs(w)
+        t = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).to(dev)
+             for n in ("q", "k", "v")}
+        t.update({n: torch.from_numpy(inp[n]).to(dev) for n in pa.GAMMA_NAMES})
+        plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=dev)
+        ws, out = plan.new_workspace(), torch.empty_like(t["q"])
+        stream = torch.cuda.current_stream()
+        for _ in range(max(3, args.warmup)):
+            pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=w.eps)
+            pa.packed_attention(t["v"], plan, ws, out)
+        torch.cuda.synchronize()
+        K = args.steps
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        for e in evs:
+            e[0].record(stream)
+            pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=w.eps)
+            e[1].record(stream)
+            pa.packed_attention(t["v"], plan, ws, out)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        if pa.device_error() != 0:
+            raise RuntimeError("kernel reported a device-side error")
+        pro = sorted(e[0].elapsed_time(e[1]) for e in evs)[K // 2]
+        att = sorted(e[1].elapsed_time(e[2]) for e in evs)[K // 2]
+        T, H, d = w.total_tokens, w.heads, w.head_dim
+        print(json.dumps({
+            "workload": w.name, "config": cfg, "total_tokens": T, "heads": H, "head_dim": d,
+            "gflop": w.flops / 1e9, "median_ms_prologue": pro, "median_ms_attention": att,
+            "tflops_step": w.flops / ((pro + att) / 1e3) / 1e12,
+            "tflops_attention": w.flops / (att / 1e3) / 1e12,
+            "frac_sustained_peak_attention": w.flops / (att / 1e3) / 1e12 /
+            float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])),
+            "tokens_per_s": T / ((pro + att) / 1e3),
+            "prologue_gbs": 8 * T * H * d / (pro / 1e3) / 1e9,
+            "peaks": peak_src}), flush=True)
+
+
 def main():
     args = parse_args()
     from packed_attention_b200.workloads import WORKLOADS, make_inputs
-    w = WORKLOADS[args.config]
+    if args.config == "all":
+        report_all(args)
+        return
+    w = WORKLOADS[int(args.config)]
     if args.impl == "reference":
         run_reference(args, w)
         return

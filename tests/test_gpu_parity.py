@@ -8,6 +8,9 @@ configuration the benchmark times and are compared on sampled rows (every
 segment's first and last rows, tile boundaries, ragged tails and random
 rows).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -150,6 +153,11 @@ def test_full_size_config_sampled_rows(cuda_device, cfg):
     ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
     got = got_all.reshape(-1, w.head_dim)[rows]
     max_abs, rel_rms = errors(got, ref)
+    report = os.environ.get("MF_PARITY_REPORT")  # optional: append the figures to a JSON-lines file
+    if report:
+        with open(report, "a") as f:
+            f.write(json.dumps({"config": cfg, "workload": w.name, "rows": int(len(rows)),
+                                "max_abs": max_abs, "rel_rms": rel_rms}) + "\n")
     assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
 
 
