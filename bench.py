@@ -35,7 +35,7 @@ KERNEL_SOURCE = os.path.join(ROOT, "packed_attention_b200", "csrc", "packed_atte
 # the full workload (profiles/traffic_packed_attention_kernel_*.md), keyed by
 # the kernel source it was taken on: any other source reports null.
 MEASURED_TRAFFIC = {
-    ("faf40727676a6f43", "hires_2048sq_4to1"): 397_379_328 + 109_314_304,
+    ("d5669df58f820a2b", "hires_2048sq_4to1"): 394_461_696 + 109_198_080,
 }
 
 
@@ -224,49 +224,97 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def report_all(args):
-    """One JSON line per workload: device time of both stages, TFLOP/s, tokens/s,
-    fraction of the measured peaks (single GPU)."""
+def _device_inputs(inp, dev, pa, torch):
+    t = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).to(dev)
+         for n in ("q", "k", "v")}
+    t.update({n: torch.from_numpy(inp[n]).to(dev) for n in pa.GAMMA_NAMES})
+    return t
+
+
+def _median_step_ms(runs, steps, warmup):
+    """Median device time (ms) per step of each stage. ``runs`` is a list of
+    (tensors, plan, workspace, out, eps, frame_dims); one step launches every
+    run's prologue and attention in order, with an event between stages."""
     import torch
     import packed_attention_b200 as pa
-    from packed_attention_b200.workloads import WORKLOADS, make_inputs
+    stream = torch.cuda.current_stream()
+
+    def launch(evs=None):
+        for i, (t, plan, ws, out, eps, frame_dims) in enumerate(runs):
+            pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=eps, frame_dims=frame_dims)
+            if evs:
+                evs[2 * i + 1].record(stream)
+            pa.packed_attention(t["v"], plan, ws, out)
+            if evs:
+                evs[2 * i + 2].record(stream)
+
+    for _ in range(max(3, warmup)):
+        launch()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(runs) + 1)]
+           for _ in range(steps)]
+    for e in evs:
+        e[0].record(stream)
+        launch(e)
+    torch.cuda.synchronize()
+    if pa.device_error() != 0:
+        raise RuntimeError("kernel reported a device-side error")
+    med = lambda xs: sorted(xs)[len(xs) // 2]
+    total = med([e[0].elapsed_time(e[-1]) for e in evs])
+    pro = med([sum(e[2 * i].elapsed_time(e[2 * i + 1]) for i in range(len(runs))) for e in evs])
+    att = med([sum(e[2 * i + 1].elapsed_time(e[2 * i + 2]) for i in range(len(runs))) for e in evs])
+    return total, pro, att
+
+
+def report_all(args):
+    """One JSON line per workload: device time of both stages, TFLOP/s, tokens/s,
+    fraction of the measured peaks (single GPU). Then one line per packed-CFG
+    pack: the pack in one forward against its two branches in two forwards."""
+    import torch
+    import packed_attention_b200 as pa
+    from packed_attention_b200.workloads import CFG_PACKS, EXTRA_WORKLOADS, WORKLOADS, make_inputs
     peaks, peak_src = load_peaks()
+    sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     dev = torch.device("cuda", 0)
-    for cfg, w in WORKLOADS.items():
-        inp = make_inputs(w)
-        t = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).to(dev)
-             for n in ("q", "k", "v")}
-        t.update({n: torch.from_numpy(inp[n]).to(dev) for n in pa.GAMMA_NAMES})
+
+    def prepare(w, inp):
+        t = _device_inputs(inp, dev, pa, torch)
         plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=dev)
-        ws, out = plan.new_workspace(), torch.empty_like(t["q"])
-        stream = torch.cuda.current_stream()
-        for _ in range(max(3, args.warmup)):
-            pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=w.eps)
-            pa.packed_attention(t["v"], plan, ws, out)
-        torch.cuda.synchronize()
-        K = args.steps
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-        for e in evs:
-            e[0].record(stream)
-            pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=w.eps)
-            e[1].record(stream)
-            pa.packed_attention(t["v"], plan, ws, out)
-            e[2].record(stream)
-        torch.cuda.synchronize()
-        if pa.device_error() != 0:
-            raise RuntimeError("kernel reported a device-side error")
-        pro = sorted(e[0].elapsed_time(e[1]) for e in evs)[K // 2]
-        att = sorted(e[1].elapsed_time(e[2]) for e in evs)[K // 2]
+        return (t, plan, plan.new_workspace(), torch.empty_like(t["q"]), w.eps, w.rope_frame_dims)
+
+    for cfg, w in list(WORKLOADS.items()) + list(EXTRA_WORKLOADS.items()):
+        _, pro, att = _median_step_ms([prepare(w, make_inputs(w))], args.steps, args.warmup)
         T, H, d = w.total_tokens, w.heads, w.head_dim
         print(json.dumps({
             "workload": w.name, "config": cfg, "total_tokens": T, "heads": H, "head_dim": d,
             "gflop": w.flops / 1e9, "median_ms_prologue": pro, "median_ms_attention": att,
             "tflops_step": w.flops / ((pro + att) / 1e3) / 1e12,
             "tflops_attention": w.flops / (att / 1e3) / 1e12,
-            "frac_sustained_peak_attention": w.flops / (att / 1e3) / 1e12 /
-            float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])),
+            "frac_sustained_peak_attention": w.flops / (att / 1e3) / 1e12 / sustained,
             "tokens_per_s": T / ((pro + att) / 1e3),
             "prologue_gbs": 8 * T * H * d / (pro / 1e3) / 1e9,
+            "rope_frame_dims": w.rope_frame_dims, "peaks": peak_src}), flush=True)
+
+    for name, cp in CFG_PACKS.items():
+        w = cp.packed()
+        inp = make_inputs(w)
+        packed = _median_step_ms([prepare(w, inp)], args.steps, args.warmup)
+        branches = []
+        for b in ("cond", "uncond"):
+            tok = cp.branch_tokens(b)
+            sub = {n: np.ascontiguousarray(inp[n][tok]) for n in ("q", "k", "v")}
+            sub.update({n: inp[n] for n in pa.GAMMA_NAMES})
+            branches.append(prepare(cp.branch(b), sub))
+        separate = _median_step_ms(branches, args.steps, args.warmup)
+        print(json.dumps({
+            "workload": name, "total_tokens": w.total_tokens, "heads": w.heads,
+            "head_dim": w.head_dim, "gflop": w.flops / 1e9,
+            "packed_ms": {"step": packed[0], "prologue": packed[1], "attention": packed[2]},
+            "two_calls_ms": {"step": separate[0], "prologue": separate[1],
+                             "attention": separate[2]},
+            "speedup_step": separate[0] / packed[0],
+            "speedup_attention": separate[2] / packed[2],
+            "tflops_attention_packed": w.flops / (packed[2] / 1e3) / 1e12,
             "peaks": peak_src}), flush=True)
 
 

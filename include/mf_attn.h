@@ -25,6 +25,7 @@
  *  - 2D RoPE, after the norm, image tokens only: grid row r rotates dims
  *    [0, d/2), grid column c rotates dims [d/2, d), in adjacent pairs
  *    (2j, 2j+1) by pos * 10000^(-2j/(d/2)). Text tokens are not rotated.
+ *    The *_3d entry points add a frame axis (see there).
  *  - Attention: non-causal softmax(q_hat k_hat^T * scale) v within a sample.
  *
  * Conventions for every entry point:
@@ -173,6 +174,43 @@ mf_status mf_joint_attn_fwd(const void* q, const void* k, const void* v, const f
                             int32_t total_tokens, int32_t heads, int32_t head_dim, float eps,
                             float softmax_scale, void* out, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/*
+ * mf_qk_prologue_3d, mf_joint_attn_fwd_3d -- the same two calls with a 3D
+ * rotary embedding: a frame axis next to the grid row and column, so that
+ * the frames of an editing sample (target, then source) are told apart by
+ * position [Mage-Flow paper summary, "Native-Resolution MMDiT (NR-MMDiT)",
+ * Conditioning: source image latents are concatenated with the target
+ * latents under a 3D RoPE with a frame dimension].
+ * Reading (the pages give no split of head_dim among the axes): dims
+ * [0, frame_dims) rotate by the token's frame index f (the sample's grids
+ * counted from 0: target 0, source 1), then two parts of
+ * S = (head_dim - frame_dims) / 2 dims rotate by the grid row r and by the
+ * grid column c. Each part rotates its adjacent pairs (2j, 2j+1) by
+ * pos * 10000^(-2j / width), width being that part's number of dims
+ * (frame_dims or S). Text tokens are not rotated. frame_dims = 0 is the 2D
+ * rotation of mf_qk_prologue / mf_joint_attn_fwd, bit for bit.
+ *   frame_dims  a multiple of 4 with 0 <= frame_dims <= head_dim - 4
+ *               (so that every part holds whole pairs); otherwise
+ *               MF_ERR_INVALID_ARG.
+ * Every other argument, and the errors, as for mf_qk_prologue and
+ * mf_joint_attn_fwd.
+ */
+mf_status mf_qk_prologue_3d(const void* q, const void* k, const float* g_q_text,
+                            const float* g_q_img, const float* g_k_text, const float* g_k_img,
+                            const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                            int32_t n_samples, int32_t total_tokens, int32_t heads,
+                            int32_t head_dim, float eps, int32_t frame_dims, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+mf_status mf_joint_attn_fwd_3d(const void* q, const void* k, const void* v,
+                               const float* g_q_text, const float* g_q_img,
+                               const float* g_k_text, const float* g_k_img,
+                               const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                               int32_t n_samples, const mf_work_item* work_dev, int32_t n_work,
+                               int32_t total_tokens, int32_t heads, int32_t head_dim, float eps,
+                               int32_t frame_dims, float softmax_scale, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * mf_joint_attn_fwd_static_scratch -- the same forward for callers that

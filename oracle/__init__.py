@@ -47,13 +47,14 @@ def _load():
             lib.oracle_total_tokens.restype = i64
             lib.oracle_total_tokens.argtypes = [i32, P, P, P, P]
             lib.oracle_qk_prologue.restype = i32
-            lib.oracle_qk_prologue.argtypes = [P, i64, i32, i32, P, P, i32, P, P, P, P, dbl, P]
+            lib.oracle_qk_prologue.argtypes = [P, i64, i32, i32, P, P, i32, P, P, P, P, dbl, i32,
+                                               P]
             lib.oracle_joint_attn.restype = i32
             lib.oracle_joint_attn.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, i32, i32, dbl,
-                                              dbl, i64, P, P, i32]
+                                              i32, dbl, i64, P, P, i32]
             lib.oracle_dense_attn.restype = i32
             lib.oracle_dense_attn.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, i32, i32, dbl,
-                                              dbl, P]
+                                              i32, dbl, P]
             _lib = lib
     return _lib
 
@@ -81,15 +82,17 @@ def total_tokens(samples) -> int:
     return int(_load().oracle_total_tokens(n, _ptr(nt), _ptr(gh), _ptr(gw), _ptr(fr)))
 
 
-def qk_prologue(x_bits, samples, g_text, g_img, eps=1e-6):
-    """Normalised, rotated q or k as fp64 ``[T, H, d]`` from bf16 bits ``[T, H, d]``."""
+def qk_prologue(x_bits, samples, g_text, g_img, eps=1e-6, frame_dims=0):
+    """Normalised, rotated q or k as fp64 ``[T, H, d]`` from bf16 bits ``[T, H, d]``.
+
+    ``frame_dims`` > 0 selects the 3D rotation (frame, row, column)."""
     x = _u16(x_bits)
     T, H, d = x.shape
     n, nt, gh, gw, fr = _samples(samples)
     out = np.empty((T, H, d), dtype=np.float64)
     gt, gi = _f32(g_text), _f32(g_img)
     rc = _load().oracle_qk_prologue(_ptr(x), T, H, d, _ptr(gt), _ptr(gi), n, _ptr(nt), _ptr(gh),
-                                    _ptr(gw), _ptr(fr), float(eps), _ptr(out))
+                                    _ptr(gw), _ptr(fr), float(eps), int(frame_dims), _ptr(out))
     if rc != 0:
         raise ValueError("oracle_qk_prologue rejected its arguments")
     return out
@@ -103,7 +106,8 @@ def _attn_args(q, k, v, gammas, samples):
     return q, k, v, g, _samples(samples)
 
 
-def joint_attn(q, k, v, gammas, samples, eps=1e-6, scale=None, rows=None, n_threads=0):
+def joint_attn(q, k, v, gammas, samples, eps=1e-6, scale=None, rows=None, n_threads=0,
+               frame_dims=0):
     """Attention output, fp64.
 
     ``rows`` (optional, int64) selects flat rows ``token * H + head``; the
@@ -121,14 +125,15 @@ def joint_attn(q, k, v, gammas, samples, eps=1e-6, scale=None, rows=None, n_thre
         out = np.empty((len(rp), d), dtype=np.float64)
         n_rows = len(rp)
     rc = _load().oracle_joint_attn(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in g], n, _ptr(nt),
-                                   _ptr(gh), _ptr(gw), _ptr(fr), H, d, float(eps), float(scale),
-                                   n_rows, _ptr(rp), _ptr(out), int(n_threads))
+                                   _ptr(gh), _ptr(gw), _ptr(fr), H, d, float(eps),
+                                   int(frame_dims), float(scale), n_rows, _ptr(rp), _ptr(out),
+                                   int(n_threads))
     if rc != 0:
         raise ValueError("oracle_joint_attn rejected its arguments")
     return out
 
 
-def dense_attn(q, k, v, gammas, samples, eps=1e-6, scale=None):
+def dense_attn(q, k, v, gammas, samples, eps=1e-6, scale=None, frame_dims=0):
     """Brute-force dense formulation (small packs only), fp64 ``[T, H, d]``."""
     q, k, v, g, (n, nt, gh, gw, fr) = _attn_args(q, k, v, gammas, samples)
     T, H, d = q.shape
@@ -136,8 +141,8 @@ def dense_attn(q, k, v, gammas, samples, eps=1e-6, scale=None):
         scale = 1.0 / np.sqrt(d)
     out = np.empty((T, H, d), dtype=np.float64)
     rc = _load().oracle_dense_attn(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in g], n, _ptr(nt),
-                                   _ptr(gh), _ptr(gw), _ptr(fr), H, d, float(eps), float(scale),
-                                   _ptr(out))
+                                   _ptr(gh), _ptr(gw), _ptr(fr), H, d, float(eps),
+                                   int(frame_dims), float(scale), _ptr(out))
     if rc != 0:
         raise ValueError("oracle_dense_attn rejected its arguments")
     return out

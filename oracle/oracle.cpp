@@ -31,6 +31,15 @@
 //   Text tokens are not rotated. Norm first, then rotation. Every frame of a
 //   multi-grid sample (an editing target and its reference image) uses the
 //   same grid positions.
+// * 3D RoPE with a frame axis, for editing samples whose source latents are
+//   concatenated with the target latents [summary, "Native-Resolution MMDiT",
+//   Conditioning: a 3D RoPE whose frame dimension tells source from target].
+//   Reading adopted (the pages give no split of head_dim): with frame_dims =
+//   F > 0, dims [0, F) rotate by the frame index f (the sample's grids counted
+//   from 0), dims [F, F + S) by r and dims [F + S, d) by c, S = (d - F) / 2;
+//   each part pairs its own dims (first + 2j, first + 2j + 1) and turns pair j
+//   by pos * 10000^(-2j / width), width being the part's size. F = 0 is the
+//   2D rotation above (parts of width d/2 for r and c).
 // * Joint self-attention confined to each sample [summary, "Native-Resolution
 //   MMDiT": FlashAttention with per-sample cumulative offsets]: for query t in
 //   sample i, s_u = (q_hat_t . k_hat_u) * scale over u in [s_i, s_i + L_i),
@@ -99,24 +108,32 @@ size_t segment_of(const std::vector<Segment>& segs, int64_t t) {
   return lo;
 }
 
-// Modality and grid position of token t of segment s.
-void token_position(const Segment& s, int64_t t, bool& is_text, int64_t& r, int64_t& c) {
+// Modality, frame and grid position of token t of segment s.
+void token_position(const Segment& s, int64_t t, bool& is_text, int64_t& f, int64_t& r,
+                    int64_t& c) {
   int64_t j = t - s.start;
   if (j < s.n_text) {
     is_text = true;
-    r = c = 0;
+    f = r = c = 0;
     return;
   }
   int64_t p = j - s.n_text;
+  f = p / (s.grid_h * s.grid_w);
   int64_t in_frame = p % (s.grid_h * s.grid_w);  // every frame shares the grid positions
   r = in_frame / s.grid_w;
   c = in_frame % s.grid_w;
   is_text = false;
 }
 
-// RMSNorm with the modality's gamma, then 2D rotation for image tokens.
-void norm_rotate(const uint16_t* x, int d, const float* gamma, bool is_text, int64_t r, int64_t c,
-                 double eps, double* out) {
+bool valid_frame_dims(int d, int frame_dims) {
+  return frame_dims >= 0 && frame_dims % 4 == 0 && frame_dims <= d - 4;
+}
+
+// RMSNorm with the modality's gamma, then the rotation for image tokens:
+// consecutive parts of head_dim for the frame (frame_dims wide, possibly
+// empty), the grid row and the grid column.
+void norm_rotate(const uint16_t* x, int d, const float* gamma, bool is_text, int64_t f, int64_t r,
+                 int64_t c, int frame_dims, double eps, double* out) {
   double sum_sq = 0.0;
   for (int m = 0; m < d; ++m) {
     double v = bf16_value(x[m]);
@@ -125,13 +142,16 @@ void norm_rotate(const uint16_t* x, int d, const float* gamma, bool is_text, int
   double inv_rms = 1.0 / std::sqrt(sum_sq / d + eps);
   for (int m = 0; m < d; ++m) out[m] = bf16_value(x[m]) * inv_rms * static_cast<double>(gamma[m]);
   if (is_text) return;
-  const int half = d / 2;
-  for (int j = 0; j < half / 2; ++j) {
-    double theta = std::pow(10000.0, -2.0 * j / half);
-    for (int axis = 0; axis < 2; ++axis) {
-      double phi = static_cast<double>(axis == 0 ? r : c) * theta;
+  const int spatial = (d - frame_dims) / 2;
+  const int first[3] = {0, frame_dims, frame_dims + spatial};
+  const int width[3] = {frame_dims, spatial, spatial};
+  const int64_t pos[3] = {f, r, c};
+  for (int axis = 0; axis < 3; ++axis) {
+    for (int j = 0; j < width[axis] / 2; ++j) {
+      double theta = std::pow(10000.0, -2.0 * j / width[axis]);
+      double phi = static_cast<double>(pos[axis]) * theta;
       double cs = std::cos(phi), sn = std::sin(phi);
-      int i0 = axis * half + 2 * j;
+      int i0 = first[axis] + 2 * j;
       double a = out[i0], b = out[i0 + 1];
       out[i0] = a * cs - b * sn;
       out[i0 + 1] = a * sn + b * cs;
@@ -156,7 +176,7 @@ struct Job {
 
 extern "C" {
 
-int oracle_abi_version() { return 1; }
+int oracle_abi_version() { return 2; }
 
 // Total tokens of the pack, or -1 if a sample is invalid.
 int64_t oracle_total_tokens(int n, const int32_t* n_text, const int32_t* grid_h,
@@ -171,19 +191,21 @@ int64_t oracle_total_tokens(int n, const int32_t* n_text, const int32_t* grid_h,
 int oracle_qk_prologue(const uint16_t* x, int64_t total_tokens, int heads, int d,
                        const float* g_text, const float* g_img, int n, const int32_t* n_text,
                        const int32_t* grid_h, const int32_t* grid_w, const int32_t* frames,
-                       double eps, double* out) {
+                       double eps, int frame_dims, double* out) {
   std::vector<Segment> segs;
   int64_t total = 0;
   if (!make_segments(n, n_text, grid_h, grid_w, frames, segs, total)) return -1;
   if (total != total_tokens || heads < 1 || d < 4 || d % 4 != 0) return -1;
+  if (!valid_frame_dims(d, frame_dims)) return -1;
   for (int64_t t = 0; t < total; ++t) {
     const Segment& s = segs[segment_of(segs, t)];
     bool is_text;
-    int64_t r, c;
-    token_position(s, t, is_text, r, c);
+    int64_t f, r, c;
+    token_position(s, t, is_text, f, r, c);
     for (int h = 0; h < heads; ++h) {
       int64_t row = t * heads + h;
-      norm_rotate(x + row * d, d, is_text ? g_text : g_img, is_text, r, c, eps, out + row * d);
+      norm_rotate(x + row * d, d, is_text ? g_text : g_img, is_text, f, r, c, frame_dims, eps,
+                  out + row * d);
     }
   }
   return 0;
@@ -196,12 +218,13 @@ int oracle_joint_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       const float* gq_text, const float* gq_img, const float* gk_text,
                       const float* gk_img, int n, const int32_t* n_text, const int32_t* grid_h,
                       const int32_t* grid_w, const int32_t* frames, int heads, int d, double eps,
-                      double scale, int64_t n_rows, const int64_t* rows, double* out,
-                      int n_threads) {
+                      int frame_dims, double scale, int64_t n_rows, const int64_t* rows,
+                      double* out, int n_threads) {
   std::vector<Segment> segs;
   int64_t total = 0;
   if (!make_segments(n, n_text, grid_h, grid_w, frames, segs, total)) return -1;
   if (heads < 1 || d < 4 || d % 4 != 0) return -1;
+  if (!valid_frame_dims(d, frame_dims)) return -1;
   if (!rows) n_rows = total * heads;
   if (n_rows < 0) return -1;
 
@@ -249,20 +272,20 @@ int oracle_joint_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
       for (int64_t u = 0; u < s.len; ++u) {
         int64_t t = s.start + u;
         bool is_text;
-        int64_t r, c;
-        token_position(s, t, is_text, r, c);
+        int64_t f, r, c;
+        token_position(s, t, is_text, f, r, c);
         int64_t row = t * heads + h;
-        norm_rotate(k + row * d, d, is_text ? gk_text : gk_img, is_text, r, c, eps,
+        norm_rotate(k + row * d, d, is_text ? gk_text : gk_img, is_text, f, r, c, frame_dims, eps,
                     &k_hat[static_cast<size_t>(u) * d]);
         for (int m = 0; m < d; ++m) v_val[static_cast<size_t>(u) * d + m] = bf16_value(v[row * d + m]);
       }
       for (size_t qi = 0; qi < job.tokens.size(); ++qi) {
         int64_t t = job.tokens[qi];
         bool is_text;
-        int64_t r, c;
-        token_position(s, t, is_text, r, c);
-        norm_rotate(q + (t * heads + h) * d, d, is_text ? gq_text : gq_img, is_text, r, c, eps,
-                    q_hat.data());
+        int64_t f, r, c;
+        token_position(s, t, is_text, f, r, c);
+        norm_rotate(q + (t * heads + h) * d, d, is_text ? gq_text : gq_img, is_text, f, r, c,
+                    frame_dims, eps, q_hat.data());
         // Pass 1: scores and their maximum.
         double mx = -std::numeric_limits<double>::infinity();
         for (int64_t u = 0; u < s.len; ++u) {
@@ -303,17 +326,19 @@ int oracle_dense_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       const float* gq_text, const float* gq_img, const float* gk_text,
                       const float* gk_img, int n, const int32_t* n_text, const int32_t* grid_h,
                       const int32_t* grid_w, const int32_t* frames, int heads, int d, double eps,
-                      double scale, double* out) {
+                      int frame_dims, double scale, double* out) {
   if (n < 1 || heads < 1 || d < 4 || d % 4 != 0) return -1;
+  if (!valid_frame_dims(d, frame_dims)) return -1;
   std::vector<int> sample_id;
   std::vector<int> text_flag;
-  std::vector<int64_t> pos_r, pos_c;
+  std::vector<int64_t> pos_f, pos_r, pos_c;
   for (int i = 0; i < n; ++i) {
     int f_count = frames ? frames[i] : 1;
     if (n_text[i] < 0 || grid_h[i] < 1 || grid_w[i] < 1 || f_count < 1) return -1;
     for (int j = 0; j < n_text[i]; ++j) {
       sample_id.push_back(i);
       text_flag.push_back(1);
+      pos_f.push_back(0);
       pos_r.push_back(0);
       pos_c.push_back(0);
     }
@@ -322,6 +347,7 @@ int oracle_dense_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
         for (int c = 0; c < grid_w[i]; ++c) {
           sample_id.push_back(i);
           text_flag.push_back(0);
+          pos_f.push_back(f);
           pos_r.push_back(r);
           pos_c.push_back(c);
         }
@@ -333,10 +359,10 @@ int oracle_dense_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     for (int64_t t = 0; t < T; ++t) {
       int64_t row = t * heads + h;
       bool txt = text_flag[t] != 0;
-      norm_rotate(q + row * d, d, txt ? gq_text : gq_img, txt, pos_r[t], pos_c[t], eps,
-                  &qh[static_cast<size_t>(t) * d]);
-      norm_rotate(k + row * d, d, txt ? gk_text : gk_img, txt, pos_r[t], pos_c[t], eps,
-                  &kh[static_cast<size_t>(t) * d]);
+      norm_rotate(q + row * d, d, txt ? gq_text : gq_img, txt, pos_f[t], pos_r[t], pos_c[t],
+                  frame_dims, eps, &qh[static_cast<size_t>(t) * d]);
+      norm_rotate(k + row * d, d, txt ? gk_text : gk_img, txt, pos_f[t], pos_r[t], pos_c[t],
+                  frame_dims, eps, &kh[static_cast<size_t>(t) * d]);
     }
     for (int64_t t = 0; t < T; ++t)
       for (int64_t u = 0; u < T; ++u) {

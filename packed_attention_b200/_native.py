@@ -56,9 +56,12 @@ SIGNATURES = {
     "mf_pack_plan": (I32, [I32, P, P, P, P, I32, I32, I64, P, P, P, P, P]),
     "mf_workspace_bytes": (SZ, [I32, I32, I32]),
     "mf_qk_prologue": (I32, [P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, P, SZ, P]),
+    "mf_qk_prologue_3d": (I32, [P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, I32, P, SZ, P]),
     "mf_packed_attention": (I32, [P, P, I32, P, I32, I32, I32, I32, F32, P, P, SZ, P]),
     "mf_joint_attn_fwd": (I32, [P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, F32, F32, P,
                                 P, SZ, P]),
+    "mf_joint_attn_fwd_3d": (I32, [P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, F32, I32,
+                                   F32, P, P, SZ, P]),
     "mf_joint_attn_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32,
                                                I32, F32, F32, P, P]),
     "mf_selftest_exp2": (I32, [P, P, I32, P]),

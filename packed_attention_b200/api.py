@@ -82,13 +82,18 @@ def _gammas(gammas, plan):
 
 
 def qk_prologue(q, k, gammas, plan: PackedPlan, workspace: torch.Tensor, eps: float = 1e-6,
-                stream=None):
+                stream=None, frame_dims: int = 0):
+    """Stage 1 into ``workspace``. ``frame_dims`` > 0 selects the 3D rotation
+    (frame, row, column) of ``mf_qk_prologue_3d``; 0 is the 2D one."""
     _check_qkv(plan, q, k)
     gs = _gammas(gammas, plan)
-    check("mf_qk_prologue", lib().mf_qk_prologue(
-        _ptr(q), _ptr(k), *[_ptr(g) for g in gs], _ptr(plan.cu_seqlens), _ptr(plan.segs),
-        plan.n_samples, plan.total_tokens, plan.heads, plan.head_dim, float(eps), _ptr(workspace),
-        workspace.numel(), _stream_handle(stream)))
+    args = [_ptr(q), _ptr(k), *[_ptr(g) for g in gs], _ptr(plan.cu_seqlens), _ptr(plan.segs),
+            plan.n_samples, plan.total_tokens, plan.heads, plan.head_dim, float(eps)]
+    tail = [_ptr(workspace), workspace.numel(), _stream_handle(stream)]
+    if frame_dims:
+        check("mf_qk_prologue_3d", lib().mf_qk_prologue_3d(*args, int(frame_dims), *tail))
+    else:
+        check("mf_qk_prologue", lib().mf_qk_prologue(*args, *tail))
 
 
 def packed_attention(v, plan: PackedPlan, workspace: torch.Tensor, out: torch.Tensor,
@@ -102,11 +107,13 @@ def packed_attention(v, plan: PackedPlan, workspace: torch.Tensor, out: torch.Te
 
 def joint_attention(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
                     softmax_scale: float = 0.0, out: torch.Tensor | None = None,
-                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                    workspace: torch.Tensor | None = None, stream=None,
+                    frame_dims: int = 0) -> torch.Tensor:
     """Packed joint text+image attention forward on device tensors.
 
     q, k, v: bf16 [T, H, d] CUDA tensors; gammas: dict of the four fp32 [d]
     CUDA tensors (g_q_text, g_q_img, g_k_text, g_k_img). Returns bf16 [T, H, d].
+    ``frame_dims`` > 0 selects the 3D rotation (``mf_joint_attn_fwd_3d``).
     """
     _check_qkv(plan, q, k, v)
     gs = _gammas(gammas, plan)
@@ -115,17 +122,22 @@ def joint_attention(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
     _check_qkv(plan, out)
     if workspace is None:
         workspace = plan.new_workspace()
-    check("mf_joint_attn_fwd", lib().mf_joint_attn_fwd(
-        _ptr(q), _ptr(k), _ptr(v), *[_ptr(g) for g in gs], _ptr(plan.cu_seqlens),
-        _ptr(plan.segs), plan.n_samples, _ptr(plan.work), plan.n_work, plan.total_tokens,
-        plan.heads, plan.head_dim, float(eps), float(softmax_scale), _ptr(out), _ptr(workspace),
-        workspace.numel(), _stream_handle(stream)))
+    head = [_ptr(q), _ptr(k), _ptr(v), *[_ptr(g) for g in gs], _ptr(plan.cu_seqlens),
+            _ptr(plan.segs), plan.n_samples, _ptr(plan.work), plan.n_work, plan.total_tokens,
+            plan.heads, plan.head_dim, float(eps)]
+    tail = [float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+            _stream_handle(stream)]
+    if frame_dims:
+        check("mf_joint_attn_fwd_3d", lib().mf_joint_attn_fwd_3d(*head, int(frame_dims), *tail))
+    else:
+        check("mf_joint_attn_fwd", lib().mf_joint_attn_fwd(*head, *tail))
     return out
 
 
 def joint_attention_host(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
                          softmax_scale: float = 0.0, out_host: torch.Tensor | None = None,
-                         device_buffers: dict | None = None, stream=None) -> torch.Tensor:
+                         device_buffers: dict | None = None, stream=None,
+                         frame_dims: int = 0) -> torch.Tensor:
     """Same forward on HOST tensors: copies inputs to the device, runs, copies the
     result back into ``out_host`` (pinned host memory makes the copies async).
 
@@ -147,7 +159,8 @@ def joint_attention_host(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
     if "workspace" not in b:
         b["workspace"] = plan.new_workspace()
     joint_attention(b["q"], b["k"], b["v"], {n: b[n] for n in GAMMA_NAMES}, plan, eps,
-                    softmax_scale, out=b["out"], workspace=b["workspace"], stream=stream)
+                    softmax_scale, out=b["out"], workspace=b["workspace"], stream=stream,
+                    frame_dims=frame_dims)
     if out_host is None:
         out_host = torch.empty(b["out"].shape, dtype=b["out"].dtype, pin_memory=True)
     out_host.copy_(b["out"], non_blocking=True)

@@ -117,18 +117,19 @@ extern "C" size_t mf_workspace_bytes(int32_t total_tokens, int32_t heads, int32_
   return layout(total_tokens, heads, head_dim, &w) ? w.total : 0;
 }
 
-extern "C" mf_status mf_qk_prologue(const void* q, const void* k, const float* g_q_text,
-                                    const float* g_q_img, const float* g_k_text,
-                                    const float* g_k_img, const int32_t* cu_seqlens_dev,
-                                    const mf_segment* segs_dev, int32_t n_samples,
-                                    int32_t total_tokens, int32_t heads, int32_t head_dim,
-                                    float eps, void* workspace, size_t workspace_bytes,
-                                    void* stream) {
+extern "C" mf_status mf_qk_prologue_3d(const void* q, const void* k, const float* g_q_text,
+                                       const float* g_q_img, const float* g_k_text,
+                                       const float* g_k_img, const int32_t* cu_seqlens_dev,
+                                       const mf_segment* segs_dev, int32_t n_samples,
+                                       int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                       float eps, int32_t frame_dims, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
   if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
   WorkspaceLayout w;
   if (!layout(total_tokens, heads, head_dim, &w) || n_samples < 1 || !(eps >= 0.0f) ||
       !std::isfinite(eps))
     return MF_ERR_INVALID_ARG;
+  if (frame_dims < 0 || frame_dims % 4 != 0 || frame_dims > head_dim - 4) return MF_ERR_INVALID_ARG;
   if (!q || !k || !g_q_text || !g_q_img || !g_k_text || !g_k_img || !cu_seqlens_dev || !segs_dev ||
       !workspace)
     return MF_ERR_INVALID_ARG;
@@ -148,15 +149,27 @@ extern "C" mf_status mf_qk_prologue(const void* q, const void* k, const float* g
   if (head_dim == 128) {
     mf::qk_prologue_kernel<128><<<grid, mf::kPrologueThreads, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
-        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps,
+        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims,
         reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat), counter);
   } else {
     mf::qk_prologue_kernel<64><<<grid, mf::kPrologueThreads, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
-        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps,
+        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims,
         reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat), counter);
   }
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
+}
+
+extern "C" mf_status mf_qk_prologue(const void* q, const void* k, const float* g_q_text,
+                                    const float* g_q_img, const float* g_k_text,
+                                    const float* g_k_img, const int32_t* cu_seqlens_dev,
+                                    const mf_segment* segs_dev, int32_t n_samples,
+                                    int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                    float eps, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  return mf_qk_prologue_3d(q, k, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev, segs_dev,
+                           n_samples, total_tokens, heads, head_dim, eps, 0, workspace,
+                           workspace_bytes, stream);
 }
 
 extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_dev,
@@ -210,6 +223,31 @@ extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_d
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
 }
 
+extern "C" mf_status mf_joint_attn_fwd_3d(const void* q, const void* k, const void* v,
+                                          const float* g_q_text, const float* g_q_img,
+                                          const float* g_k_text, const float* g_k_img,
+                                          const int32_t* cu_seqlens_dev,
+                                          const mf_segment* segs_dev, int32_t n_samples,
+                                          const mf_work_item* work_dev, int32_t n_work,
+                                          int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                          float eps, int32_t frame_dims, float softmax_scale,
+                                          void* out, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  // Check everything the second stage needs before launching the first.
+  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
+  if (!v || !work_dev || !out || n_work < 1 || !std::isfinite(softmax_scale))
+    return MF_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(out)) return MF_ERR_ALIGNMENT;
+  const size_t bytes = static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * heads * head_dim * 2;
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes)) return MF_ERR_INVALID_ARG;
+  mf_status st = mf_qk_prologue_3d(q, k, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev,
+                                   segs_dev, n_samples, total_tokens, heads, head_dim, eps,
+                                   frame_dims, workspace, workspace_bytes, stream);
+  if (st != MF_OK) return st;
+  return mf_packed_attention(v, segs_dev, n_samples, work_dev, n_work, total_tokens, heads,
+                             head_dim, softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
 extern "C" mf_status mf_joint_attn_fwd(const void* q, const void* k, const void* v,
                                        const float* g_q_text, const float* g_q_img,
                                        const float* g_k_text, const float* g_k_img,
@@ -218,19 +256,9 @@ extern "C" mf_status mf_joint_attn_fwd(const void* q, const void* k, const void*
                                        int32_t n_work, int32_t total_tokens, int32_t heads,
                                        int32_t head_dim, float eps, float softmax_scale, void* out,
                                        void* workspace, size_t workspace_bytes, void* stream) {
-  // Check everything the second stage needs before launching the first.
-  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
-  if (!v || !work_dev || !out || n_work < 1 || !std::isfinite(softmax_scale))
-    return MF_ERR_INVALID_ARG;
-  if (!aligned16(v) || !aligned16(out)) return MF_ERR_ALIGNMENT;
-  const size_t bytes = static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * heads * head_dim * 2;
-  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes)) return MF_ERR_INVALID_ARG;
-  mf_status st = mf_qk_prologue(q, k, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev,
-                                segs_dev, n_samples, total_tokens, heads, head_dim, eps, workspace,
-                                workspace_bytes, stream);
-  if (st != MF_OK) return st;
-  return mf_packed_attention(v, segs_dev, n_samples, work_dev, n_work, total_tokens, heads,
-                             head_dim, softmax_scale, out, workspace, workspace_bytes, stream);
+  return mf_joint_attn_fwd_3d(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev,
+                              segs_dev, n_samples, work_dev, n_work, total_tokens, heads, head_dim,
+                              eps, 0, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
 namespace {

@@ -16,10 +16,10 @@
 //                    load the S row from TMEM, mask keys past the sample
 //                    end, online max and sum in the exp2 domain, write P
 //                    (bf16) back into TMEM over S, and rescale O in TMEM only
-//                    when the running max grew by more than 2^8 (a stale max
-//                    keeps p <= 256: exact enough in bf16, safe in fp32). At
-//                    the end of an item: O / l -> bf16 rows, skipping rows
-//                    past the sample end.
+//                    when the running max of a row inside the sample grew by
+//                    more than 2^8 (a stale max keeps p <= 256: exact enough
+//                    in bf16, safe in fp32). At the end of an item: O / l ->
+//                    bf16 rows, skipping rows past the sample end.
 //   warp 8 (1 lane)  TMA producer: both Q sub-tiles per item, then K_j, V_j
 //                    into a ring of shared-memory stages (128-byte swizzled
 //                    boxes of 128 rows x 64 dims).
@@ -429,6 +429,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
       const ItemInfo it = load_item(p, idx);
       if (t == 1 && !it.b_valid) continue;
+      // Rows past the sample end (another sample's tokens, or zeros) are
+      // computed but never stored, and they take no part in the rescale vote:
+      // a sample's output then depends on its own tokens only, whatever it is
+      // packed with.
+      const bool row_in = it.q0 + t * kSubM + row < it.seg_start + it.seg_len;
       float m = -INFINITY;  // running max of s * scale * log2(e)
       float l = 0.0f;       // running sum of p
       for (int j = 0; j < it.n_kv; ++j) {
@@ -461,7 +466,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mx1 = fmax3(mx1, s[126], s[127]);
         const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
         const float m_new = fmaxf(m, m_tile);
-        if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
+        if (j == 0 || __any_sync(0xffffffffu, row_in && m_new > m + kRescaleThreshold)) {
           // S_t(j) has landed, so PV_t(j-1) is complete: O_t may be rescaled.
           const float factor = ex2_approx(m - m_new);  // 0 on the first step
           l *= factor;
@@ -488,7 +493,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint64_t x = fma_f32x2(f32x2(s[e], s[e + 1]), sl2x2, neg_m);
             float x0, x1, p0, p1;
             f32x2_split(x, x0, x1);
-            if (kPolyEvery > 0 && c % kPolyEvery == kPolyEvery - 1) {
+            if (kPolyEvery > 0 && c % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
               exp2_fma_x2(x0, x1, p0, p1);  // a share of the exponentials on the FMA pipe
             } else {
               p0 = ex2_approx(x0);
@@ -513,7 +518,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ++no;
       tc_fence_after_sync();
       const int q_row = it.q0 + t * kSubM + row;
-      const bool store = q_row < it.seg_start + it.seg_len;
+      const bool store = row_in;
       const float inv_l = 1.0f / l;
       uint4* dst = reinterpret_cast<uint4*>(p.out) +
                    (static_cast<size_t>(q_row) * p.heads + it.head) * (D / 8);

@@ -17,7 +17,7 @@
 
 #include "../../include/mf_attn.h"
 
-extern "C" int32_t mf_abi_version(void) { return 1; }
+extern "C" int32_t mf_abi_version(void) { return 2; }
 
 extern "C" const char* mf_status_string(mf_status status) {
   switch (status) {

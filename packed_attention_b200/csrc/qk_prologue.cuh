@@ -11,6 +11,13 @@
 // r * theta_j and dims [d/2, d) by c * theta_j, theta_j = 10000^(-2j/(d/2)).
 // Text tokens are not rotated. All arithmetic in fp32, one bf16 rounding.
 //
+// With frame_dims = F > 0 the rotation is 3D [same section, Conditioning:
+// source and target latents told apart by a frame dimension of the RoPE]:
+// dims [0, F) rotate by the token's frame index f (the sample's grids
+// counted from 0), then two parts of S = (d - F) / 2 dims rotate by r and by
+// c; each part uses theta_j = 10000^(-2j/width) with its own width (F or S).
+// F = 0 is the 2D rotation above.
+//
 // HBM-bound: it reads q and k and writes q_hat and k_hat once (8 * T * H * d
 // bytes). Layout of the work: a group of d/8 threads owns one token and
 // loops over its heads; each thread holds 8 consecutive dims (one 16-byte
@@ -52,10 +59,11 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
     const float* __restrict__ gq_img, const float* __restrict__ gk_text,
     const float* __restrict__ gk_img, const int32_t* __restrict__ cu_seqlens,
     const mf_segment* __restrict__ segs, int n_samples, int total_tokens, int heads, float eps,
-    uint4* __restrict__ q_hat, uint4* __restrict__ k_hat, int32_t* __restrict__ work_counter) {
+    int frame_dims, uint4* __restrict__ q_hat, uint4* __restrict__ k_hat,
+    int32_t* __restrict__ work_counter) {
   constexpr int kVecPerRow = D / 8;                          // 16-byte vectors per row
   constexpr int kTokPerBlock = kPrologueThreads / kVecPerRow;
-  constexpr int kHalf = D / 2;
+  const int spatial = (D - frame_dims) / 2;  // dims per grid axis
 
   if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
 
@@ -85,11 +93,10 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
 #pragma unroll
     for (int i = 0; i < 4; ++i) { cs[i] = 1.0f; sn[i] = 0.0f; }
   } else {
+    const int frame = (j - n_text) / hw;
     const int p = (j - n_text) % hw;  // every frame of a sample shares the grid positions
-    const int axis = e0 >= kHalf;     // 0: grid row, 1: grid column
-    const int pos = axis ? p % gw : p / gw;
-    const int pair0 = (e0 - axis * kHalf) / 2;
-    // theta_j = 10000^(-2j/half) = 2^(-(2j/half) * log2(10000)). The angle
+    const int row = p / gw, col = p % gw;
+    // theta_j = 10000^(-2j/width) = 2^(-(2j/width) * log2(10000)). The angle
     // pos * theta_j is formed and reduced to [-pi, pi] in fp64 (once per token
     // and thread), so the fp32 sine and cosine see an argument accurate to
     // ~1e-7 rad however large the grid position is.
@@ -98,7 +105,16 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
     constexpr double kInvTwoPi = 0.15915494309189535;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const double theta = exp2(-(2.0 * (pair0 + i) / kHalf) * kLog2Base);
+      const int e = e0 + 2 * i;  // first dim of this pair
+      int pos, first, width;
+      if (e < frame_dims) {
+        pos = frame; first = 0; width = frame_dims;
+      } else if (e < frame_dims + spatial) {
+        pos = row; first = frame_dims; width = spatial;
+      } else {
+        pos = col; first = frame_dims + spatial; width = spatial;
+      }
+      const double theta = exp2(-(2.0 * ((e - first) / 2) / width) * kLog2Base);
       double ang = static_cast<double>(pos) * theta;
       ang -= kTwoPi * rint(ang * kInvTwoPi);
       sincosf(static_cast<float>(ang), &sn[i], &cs[i]);

@@ -37,6 +37,8 @@ class Workload:
     outlier_scale: float = 1.0
     eps: float = 1e-6
     notes: str = field(default="", compare=False)
+    # 3D RoPE: dims of head_dim that rotate by the frame index (0: 2D RoPE)
+    rope_frame_dims: int = 0
 
     @property
     def seg_lens(self):
@@ -58,7 +60,7 @@ class Workload:
     def with_heads(self, heads: int) -> "Workload":
         return Workload(self.name + f"_h{heads}", self.samples, heads, self.head_dim, self.seed,
                         self.token_budget, self.sigma_ranges, self.outlier_frac, self.outlier_scale,
-                        self.eps, self.notes)
+                        self.eps, self.notes, self.rope_frame_dims)
 
 
 WORKLOADS = {
@@ -77,6 +79,18 @@ WORKLOADS = {
     4: Workload("hires_2048sq_4to1", ((512, 128, 128, 1), (256, 32, 128, 1)), heads=24,
                 head_dim=128, seed=4, outlier_frac=0.01, outlier_scale=8.0,
                 notes="2048^2 sample (16,896 tokens) + 4:1 sample (4,352 tokens); 1% of K rows x8"),
+}
+
+# Editing with the frame axis of the RoPE: the 1024^2 edit pack, its source
+# (reference) grid told apart from the target grid by a 3D rotation (Mage-Flow
+# paper summary, "Native-Resolution MMDiT (NR-MMDiT)", Conditioning). The
+# pages give no split of head_dim; F = d/8 = 16 dims for the frame leaves 56
+# for each grid axis.
+EXTRA_WORKLOADS = {
+    "edit_1024sq_rope3d": Workload(
+        "edit_1024sq_rope3d", ((512, 64, 64, 2),), heads=24, head_dim=128, seed=3,
+        sigma_ranges=((512 + 4096, 512 + 2 * 4096, 0.5),), rope_frame_dims=16,
+        notes="the 1024^2 edit pack under 3D RoPE: 16 frame dims, 56 per grid axis"),
 }
 
 
@@ -124,3 +138,62 @@ def random_pack(rng: np.random.Generator, n_samples: int, max_text: int, max_sid
         out.append((int(rng.integers(0, max_text + 1)), int(rng.integers(1, max_side + 1)),
                     int(rng.integers(1, max_side + 1)), int(rng.integers(1, max_frames + 1))))
     return tuple(out)
+
+
+@dataclass(frozen=True)
+class CfgPack:
+    """Classifier-free guidance evaluated as one pack.
+
+    Each request contributes two samples that share its latent grid: the
+    conditional branch (its prompt's text tokens, then the grid) and the
+    unconditional branch (the empty prompt, then the same grid). Both go into
+    one pack and one forward instead of two (Mage-Flow paper summary,
+    "Native-Resolution MMDiT (NR-MMDiT)": packed CFG inference; video
+    overview, 00:04:03). The pages give no text length for the unconditional
+    branch; the empty prompt is read as ``n_text_uncond`` = 0 text tokens.
+    Samples are packed request by request: cond_0, uncond_0, cond_1, ...
+    """
+    name: str
+    requests: tuple  # of (n_text_cond, H_lat, W_lat)
+    heads: int
+    head_dim: int
+    seed: int
+    n_text_uncond: int = 0
+    notes: str = field(default="", compare=False)
+
+    def samples(self, branch=None):
+        """Samples of the whole pack (branch None), or of one branch ('cond' / 'uncond')."""
+        out = []
+        for (nt, h, w) in self.requests:
+            if branch in (None, "cond"):
+                out.append((nt, h, w, 1))
+            if branch in (None, "uncond"):
+                out.append((self.n_text_uncond, h, w, 1))
+        return tuple(out)
+
+    def packed(self) -> Workload:
+        return Workload(self.name, self.samples(), self.heads, self.head_dim, self.seed,
+                        notes=self.notes)
+
+    def branch(self, branch: str) -> Workload:
+        return Workload(f"{self.name}_{branch}", self.samples(branch), self.heads, self.head_dim,
+                        self.seed, notes=f"{branch} branch of {self.name}")
+
+    def branch_tokens(self, branch: str) -> np.ndarray:
+        """Token indices, in the packed layout, of the given branch's samples in order."""
+        idx, start = [], 0
+        for i, L in enumerate(self.packed().seg_lens):
+            if (i % 2 == 0) == (branch == "cond"):
+                idx.append(np.arange(start, start + L))
+            start += L
+        return np.concatenate(idx)
+
+
+CFG_PACKS = {
+    "cfg_1024sq": CfgPack("cfg_1024sq", ((512, 64, 64),), heads=24, head_dim=128, seed=5,
+                          notes="one 1024^2 request: cond 512 text + 64x64, uncond 64x64"),
+    "cfg_mixed_native_res": CfgPack(
+        "cfg_mixed_native_res", ((128, 32, 32), (256, 64, 64), (40, 16, 64), (200, 48, 64)),
+        heads=24, head_dim=128, seed=6,
+        notes="four requests (512^2, 1024^2, 4:1, 768x1024), each cond + uncond"),
+}

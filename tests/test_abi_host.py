@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.mf_abi_version() == 1
+    assert lib.mf_abi_version() == 2
     for code, name in _native.STATUS.items():
         assert lib.mf_status_string(code).decode() == name
 
@@ -155,6 +155,24 @@ def test_forward_argument_checks(lib):
     assert _fwd(lib, scale=float("inf")) == -1
     assert _fwd(lib, out=0x10000) == -1        # out aliases q
     assert _fwd(lib, ws=0x10000 - 0x100) == -1  # workspace overlaps q
+
+
+def test_frame_dims_checked_before_any_launch(lib):
+    """mf_joint_attn_fwd_3d / mf_qk_prologue_3d refuse a split of head_dim that
+    does not give every axis whole pairs; everything else as in the 2D call."""
+    P = ctypes.c_void_p
+    base = (P(0x10000), P(0x20000), P(0x30000), P(0x40000), P(0x40100), P(0x40200), P(0x40300),
+            P(0x50000), P(0x60000), 2, P(0x70000), 4, 152, 2, 64, 1e-6)
+    tail = (0.0, P(0x80000), P(0x100000), 1 << 20, None)
+    for F in (-4, 2, 6, 62, 64, 1000):
+        assert lib.mf_joint_attn_fwd_3d(*base, F, *tail) == -1, F
+    pro = (P(0x10000), P(0x20000), P(0x40000), P(0x40100), P(0x40200), P(0x40300), P(0x50000),
+           P(0x60000), 2, 152, 2, 128, 1e-6)
+    for F in (-4, 2, 126, 128):
+        assert lib.mf_qk_prologue_3d(*pro, F, P(0x100000), 1 << 20, None) == -1, F
+    # the shared checks still come first: unsupported head_dim, misaligned input
+    assert lib.mf_joint_attn_fwd_3d(*base[:14], 96, 1e-6, 2, *tail) == -2
+    assert lib.mf_joint_attn_fwd_3d(P(0x10008), *base[1:], 16, *tail) == -3
 
 
 def test_diagnostic_entry_points_reject_bad_arguments(lib):

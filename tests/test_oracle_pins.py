@@ -193,6 +193,144 @@ def test_rope_scores_depend_only_on_offset(d):
         assert s1 == pytest.approx(s0, abs=1e-10 * d)
 
 
+# ---------------------------------------------------- 3D RoPE (frame axis) ---
+# Reading under test: with frame_dims = F, dims [0, F) turn by the frame index
+# f, [F, F + S) by the grid row r and [F + S, d) by the column c, S = (d - F)/2;
+# pair j of a part of width w turns by pos * 10000^(-2j/w).
+
+@pytest.mark.parametrize("d,F", [(64, 8), (128, 16), (128, 32), (64, 60)])
+def test_rope3d_unit_vector_angles(d, F):
+    S = (d - F) // 2
+    H_lat, W_lat, frames = 3, 4, 3
+    samples = [(0, H_lat, W_lat, frames)]
+    T = frames * H_lat * W_lat
+    g = np.ones(d, dtype=np.float32)
+    root_d = math.sqrt(d)
+    parts = ((0, F), (F, S), (F + S, S))  # (first dim, width): frame, row, column
+    for f, r, c in ((2, 1, 3), (1, 2, 0), (0, 2, 3)):
+        t = f * H_lat * W_lat + r * W_lat + c
+        for (first, width), pos in zip(parts, (f, r, c)):
+            for j in sorted({0, min(1, width // 2 - 1), width // 2 - 1}):
+                for odd in (0, 1):
+                    m = first + 2 * j + odd
+                    x = np.zeros((T, 1, d), dtype=np.uint16)
+                    x[:, 0, m] = ONE_BF16
+                    y = oracle.qk_prologue(x, samples, g, g, eps=0.0, frame_dims=F)[t, 0]
+                    phi = pos * 10000.0 ** (-2.0 * j / width)
+                    want = (math.cos(phi), math.sin(phi)) if odd == 0 else (-math.sin(phi), math.cos(phi))
+                    i0 = first + 2 * j
+                    assert y[i0] == pytest.approx(root_d * want[0], abs=1e-12)
+                    assert y[i0 + 1] == pytest.approx(root_d * want[1], abs=1e-12)
+                    mask = np.ones(d, bool)
+                    mask[[i0, i0 + 1]] = False
+                    assert np.all(y[mask] == 0.0)
+
+
+def test_rope3d_theta_literal_values():
+    # Widths chosen so that the frequencies are powers of ten:
+    # F = 16: pair 1 turns by 10000^(-2/16) = 10^(-1/2) per frame, pair 4 by 10^-2;
+    # S = 56 (d = 128): pair 7 turns by 10000^(-14/56) = 10^-1 per row;
+    # d = 64, F = 8: frame pair 1 by 10^-1, S = 28: row pair 7 by 10^-2.
+    cases = [(128, 16, 2, 0.31622776601683794, "f"), (128, 16, 8, 0.01, "f"),
+             (128, 16, 16 + 14, 0.1, "r"), (128, 16, 16 + 56 + 14, 0.1, "c"),
+             (64, 8, 2, 0.1, "f"), (64, 8, 8 + 14, 0.01, "r")]
+    for d, F, m, theta, axis in cases:
+        samples = [(0, 2, 2, 2)]  # token 4 + (r*2 + c): frame 1
+        x = np.zeros((8, 1, d), dtype=np.uint16)
+        x[:, 0, m] = ONE_BF16
+        g = np.ones(d, dtype=np.float32)
+        y = oracle.qk_prologue(x, samples, g, g, eps=0.0, frame_dims=F)
+        # one step along the axis: frame 1 at (0, 0), frame 0 at (1, 0), frame 0 at (0, 1)
+        t = {"f": 4, "r": 2, "c": 1}[axis]
+        assert math.atan2(y[t, 0, m + 1], y[t, 0, m]) == pytest.approx(theta, abs=1e-13)
+
+
+@pytest.mark.parametrize("d,F", [(64, 8), (128, 16)])
+def test_rope3d_scores_depend_only_on_offset(d, F):
+    H_lat, W_lat, frames = 6, 6, 4
+    samples = [(0, H_lat, W_lat, frames)]
+    T = frames * H_lat * W_lat
+    qrow, krow = rand_bits(15, (1, 1, d)), rand_bits(16, (1, 1, d))
+    g = np.ones(d, dtype=np.float32)
+    qh = oracle.qk_prologue(np.repeat(qrow, T, 0), samples, g, g, frame_dims=F)[:, 0]
+    kh = oracle.qk_prologue(np.repeat(krow, T, 0), samples, g, g, frame_dims=F)[:, 0]
+
+    def tok(f, r, c):
+        return (f * H_lat + r) * W_lat + c
+
+    rng = np.random.default_rng(1)
+    seen_frame_effect = False
+    for _ in range(40):
+        f1, f2 = rng.integers(0, 2, size=2)
+        r1, c1, r2, c2 = rng.integers(0, 3, size=4)
+        a = int(rng.integers(0, 2))
+        b, c = rng.integers(0, 3, size=2)
+        s0 = qh[tok(f1, r1, c1)] @ kh[tok(f2, r2, c2)]
+        s1 = qh[tok(f1 + a, r1 + b, c1 + c)] @ kh[tok(f2 + a, r2 + b, c2 + c)]
+        assert s1 == pytest.approx(s0, abs=1e-10 * d)
+        if f1 != f2:
+            s_same = qh[tok(f1, r1, c1)] @ kh[tok(f1, r2, c2)]
+            seen_frame_effect |= abs(s_same - s0) > 1e-6
+    assert seen_frame_effect  # the frame offset does change the score
+
+
+def test_rope3d_frames_differ_only_in_frame_dims():
+    # Identical raw tokens in the target (f = 0) and source (f = 1) frames:
+    # row/column dims agree exactly, the target's frame dims are unrotated and
+    # the source's frame dims are the target's turned by theta_j.
+    d, F = 128, 16
+    samples = [(3, 4, 5, 2)]
+    x = rand_bits(96, (43, 2, d))
+    x[23:43] = x[3:23]
+    g = rand_gammas(9, d)
+    y = oracle.qk_prologue(x, samples, g["g_k_text"], g["g_k_img"], frame_dims=F)
+    y2d = oracle.qk_prologue(x, samples, g["g_k_text"], g["g_k_img"])
+    np.testing.assert_array_equal(y[23:43, :, F:], y[3:23, :, F:])
+    # the normalised values alone: every token read as text, with the image gamma
+    nrm = oracle.qk_prologue(x, [(42, 1, 1, 1)], g["g_k_img"], g["g_k_img"])
+    # target frame dims: the normalised values themselves (f = 0 is the identity)
+    np.testing.assert_allclose(y[3:23, :, :F], nrm[3:23, :, :F], rtol=0, atol=1e-15)
+    for j in range(F // 2):
+        th = 10000.0 ** (-2.0 * j / F)
+        a, b = y[3:23, :, 2 * j], y[3:23, :, 2 * j + 1]
+        np.testing.assert_allclose(y[23:43, :, 2 * j], a * math.cos(th) - b * math.sin(th), atol=1e-13)
+        np.testing.assert_allclose(y[23:43, :, 2 * j + 1], a * math.sin(th) + b * math.cos(th), atol=1e-13)
+    # text tokens are never rotated, so they agree with the 2D prologue
+    np.testing.assert_array_equal(y[:3], y2d[:3])
+
+
+def test_rope3d_preserves_norm_and_rejects_bad_splits():
+    d = 128
+    samples = [(1, 3, 4, 3)]
+    T = 1 + 36
+    row = rand_bits(17, (1, 2, d))
+    x = np.repeat(row, T, axis=0)
+    g = rand_gammas(4, d)["g_q_img"]
+    for F in (4, 16, 124):
+        y = oracle.qk_prologue(x, samples, g, g, frame_dims=F)
+        ref = np.linalg.norm(y[0], axis=-1)
+        for t in range(1, T):
+            np.testing.assert_allclose(np.linalg.norm(y[t], axis=-1), ref, rtol=1e-13)
+    for F in (-4, 2, 6, 126, 128):
+        with pytest.raises(ValueError):
+            oracle.qk_prologue(x, samples, g, g, frame_dims=F)
+
+
+@pytest.mark.parametrize("trial", range(4))
+def test_rope3d_dense_brute_force(trial):
+    rng = np.random.default_rng(700 + trial)
+    samples = random_pack(rng, int(rng.integers(1, 4)), 8, 4, 3)
+    d = (64, 128)[trial % 2]
+    F = (8, 16, 32, 4)[trial]
+    H = int(rng.integers(1, 3))
+    q, k, v, g = _pack_inputs(samples, H, d, 300 + trial)
+    a = oracle.joint_attn(q, k, v, g, samples, frame_dims=F)
+    b = oracle.dense_attn(q, k, v, g, samples, frame_dims=F)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    if any(f > 1 for (_, _, _, f) in samples):
+        assert not np.allclose(a, oracle.joint_attn(q, k, v, g, samples), atol=1e-6)
+
+
 # -------------------------------------------------------------- attention ---
 
 def _pack_inputs(samples, H, d, seed):

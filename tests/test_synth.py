@@ -4,7 +4,7 @@ import pytest
 import torch
 
 from packed_attention_b200 import synth
-from packed_attention_b200.workloads import WORKLOADS, make_inputs
+from packed_attention_b200.workloads import CFG_PACKS, WORKLOADS, make_inputs
 
 
 def test_splitmix64_known_answers():
@@ -87,3 +87,24 @@ def test_edit_reference_tokens_have_half_sigma():
     v = synth.bf16_bits_to_f64(inp["v"])
     assert abs(v[:4608].std() - 1.0) < 0.02
     assert abs(v[4608:].std() - 0.5) < 0.01
+
+
+@pytest.mark.parametrize("name", sorted(CFG_PACKS))
+def test_cfg_pack_layout(name):
+    cp = CFG_PACKS[name]
+    w = cp.packed()
+    # request by request: cond (prompt + grid), then uncond (empty prompt + same grid)
+    assert len(w.samples) == 2 * len(cp.requests)
+    for r, (nt, h, wd) in enumerate(cp.requests):
+        assert w.samples[2 * r] == (nt, h, wd, 1)
+        assert w.samples[2 * r + 1] == (cp.n_text_uncond, h, wd, 1)
+    cond, uncond = cp.branch_tokens("cond"), cp.branch_tokens("uncond")
+    # the two branches partition the pack's tokens, each in increasing order
+    both = np.sort(np.concatenate([cond, uncond]))
+    np.testing.assert_array_equal(both, np.arange(w.total_tokens))
+    assert np.all(np.diff(cond) > 0) and np.all(np.diff(uncond) > 0)
+    assert len(cond) == cp.branch("cond").total_tokens
+    assert len(uncond) == cp.branch("uncond").total_tokens
+    # the first token of each branch segment is where the pack places it
+    starts = np.concatenate([[0], np.cumsum(w.seg_lens)[:-1]])
+    assert cond[0] == starts[0] and uncond[0] == starts[1]
