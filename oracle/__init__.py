@@ -8,7 +8,9 @@ marshals numpy arrays through ctypes.
 
 Parity status: every function is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_pins.py`` (closed forms, invariants and a dense
-brute-force formulation); none is "parity unpinned".
+brute-force formulation) and, for the gradients of :func:`attn_grad`,
+``tests/test_oracle_grad_pins.py`` (central finite differences, closed forms
+and invariants); none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -52,6 +54,9 @@ def _load():
             lib.oracle_joint_attn.restype = i32
             lib.oracle_joint_attn.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, i32, i32, dbl,
                                               i32, dbl, i64, P, P, i32]
+            lib.oracle_attn_grad.restype = i32
+            lib.oracle_attn_grad.argtypes = [P, P, P, P, P, P, P, P, i32, P, P, P, P, i32, i32, dbl,
+                                             i32, dbl, P, P, P, P, P, i32]
             lib.oracle_dense_attn.restype = i32
             lib.oracle_dense_attn.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, i32, i32, dbl,
                                               i32, dbl, P]
@@ -146,3 +151,41 @@ def dense_attn(q, k, v, gammas, samples, eps=1e-6, scale=None, frame_dims=0):
     if rc != 0:
         raise ValueError("oracle_dense_attn rejected its arguments")
     return out
+
+
+def attn_grad(q, k, v, gammas, samples, dout=None, eps=1e-6, scale=None, frame_dims=0,
+              n_threads=0):
+    """Forward output and, given ``dout`` = dL/dout, the gradients, all fp64.
+
+    q, k, v, dout: float64 ``[T, H, d]`` values (not bf16 bits); gammas: dict of
+    the four ``[d]`` vectors. Returns a dict with ``out`` and, with ``dout``,
+    ``dq``, ``dk``, ``dv`` (``[T, H, d]``) and ``dgamma`` (a dict keyed like
+    the gammas).
+    """
+    q, k, v = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+    if q.shape != k.shape or q.shape != v.shape or q.ndim != 3:
+        raise ValueError("q, k, v must share one [T, H, d] shape")
+    T, H, d = q.shape
+    names = ("g_q_text", "g_q_img", "g_k_text", "g_k_img")
+    g = [np.ascontiguousarray(gammas[nm], dtype=np.float64) for nm in names]
+    n, nt, gh, gw, fr = _samples(samples)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((T, H, d), dtype=np.float64)
+    res = {"out": out}
+    go = dq = dk = dv = dg = None
+    if dout is not None:
+        go = np.ascontiguousarray(dout, dtype=np.float64)
+        if go.shape != q.shape:
+            raise ValueError("dout must have the shape of q")
+        dq, dk, dv = (np.empty((T, H, d), dtype=np.float64) for _ in range(3))
+        dg = np.empty((4, d), dtype=np.float64)
+    rc = _load().oracle_attn_grad(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in g], _ptr(go), n,
+                                  _ptr(nt), _ptr(gh), _ptr(gw), _ptr(fr), H, d, float(eps),
+                                  int(frame_dims), float(scale), _ptr(out), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(dg), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_attn_grad rejected its arguments")
+    if dout is not None:
+        res.update(dq=dq, dk=dk, dv=dv, dgamma={nm: dg[i] for i, nm in enumerate(names)})
+    return res

@@ -46,6 +46,8 @@
 //   then o_t = sum_u exp(s_u - max s) v_u / sum_u exp(s_u - max s). Non-causal.
 //   Computed in two passes (scores, then max, then the weighted sum): no
 //   online rescaling.
+// * Gradients of all of the above for training (oracle_attn_grad, at the end
+//   of the file): the chain rule written out, on fp64 inputs.
 //
 // Inputs are bf16 bit patterns converted exactly to fp64; gammas are fp32
 // values; all arithmetic is fp64.
@@ -129,6 +131,28 @@ bool valid_frame_dims(int d, int frame_dims) {
   return frame_dims >= 0 && frame_dims % 4 == 0 && frame_dims <= d - 4;
 }
 
+// Rotation of an image token's vector in place: consecutive parts of head_dim
+// for the frame (frame_dims wide, possibly empty), the grid row and the grid
+// column; pair j of a part of width w turns by pos * 10000^(-2j/w). sign = -1
+// applies the inverse (transposed) rotation.
+void rotate_pairs(double* v, int d, int frame_dims, int64_t f, int64_t r, int64_t c, double sign) {
+  const int spatial = (d - frame_dims) / 2;
+  const int first[3] = {0, frame_dims, frame_dims + spatial};
+  const int width[3] = {frame_dims, spatial, spatial};
+  const int64_t pos[3] = {f, r, c};
+  for (int axis = 0; axis < 3; ++axis) {
+    for (int j = 0; j < width[axis] / 2; ++j) {
+      double theta = std::pow(10000.0, -2.0 * j / width[axis]);
+      double phi = sign * static_cast<double>(pos[axis]) * theta;
+      double cs = std::cos(phi), sn = std::sin(phi);
+      int i0 = first[axis] + 2 * j;
+      double a = v[i0], b = v[i0 + 1];
+      v[i0] = a * cs - b * sn;
+      v[i0 + 1] = a * sn + b * cs;
+    }
+  }
+}
+
 // RMSNorm with the modality's gamma, then the rotation for image tokens:
 // consecutive parts of head_dim for the frame (frame_dims wide, possibly
 // empty), the grid row and the grid column.
@@ -142,21 +166,7 @@ void norm_rotate(const uint16_t* x, int d, const float* gamma, bool is_text, int
   double inv_rms = 1.0 / std::sqrt(sum_sq / d + eps);
   for (int m = 0; m < d; ++m) out[m] = bf16_value(x[m]) * inv_rms * static_cast<double>(gamma[m]);
   if (is_text) return;
-  const int spatial = (d - frame_dims) / 2;
-  const int first[3] = {0, frame_dims, frame_dims + spatial};
-  const int width[3] = {frame_dims, spatial, spatial};
-  const int64_t pos[3] = {f, r, c};
-  for (int axis = 0; axis < 3; ++axis) {
-    for (int j = 0; j < width[axis] / 2; ++j) {
-      double theta = std::pow(10000.0, -2.0 * j / width[axis]);
-      double phi = static_cast<double>(pos[axis]) * theta;
-      double cs = std::cos(phi), sn = std::sin(phi);
-      int i0 = first[axis] + 2 * j;
-      double a = out[i0], b = out[i0 + 1];
-      out[i0] = a * cs - b * sn;
-      out[i0 + 1] = a * sn + b * cs;
-    }
-  }
+  rotate_pairs(out, d, frame_dims, f, r, c, 1.0);
 }
 
 int resolve_threads(int n_threads) {
@@ -388,6 +398,203 @@ int oracle_dense_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
         double a = 0.0;
         for (int64_t u = 0; u < T; ++u) a += srow[u] * bf16_value(v[(u * heads + h) * d + m]);
         o[m] = a / denom;
+      }
+    }
+  }
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
+// Gradients, for training. The pages' headline speedup is for training the
+// NR-MMDiT [video overview, 00:05:08; summary, "Training Infrastructure"], so
+// the path's backward is the derivative of the forward above, by the chain
+// rule, for a loss L with dL/dout = G:
+//   P_tu = exp(s_tu - M_t) / Z_t, s_tu = scale * q_hat_t . k_hat_u   (within a sample)
+//   dv_u     = sum_t P_tu G_t
+//   dP_tu    = G_t . v_u,  D_t = sum_u P_tu dP_tu,  dS_tu = P_tu (dP_tu - D_t)
+//   dq_hat_t = scale * sum_u dS_tu k_hat_u,  dk_hat_u = scale * sum_t dS_tu q_hat_t
+//   dy       = R(pos)^T dx_hat                      (rotation transposed; text: dy = dx_hat)
+//   dgamma  += dy * x_n                              (per role and modality, summed over tokens and heads)
+//   dx       = r * (dx_n - x_n * (x_n . dx_n) / d),  dx_n = dy * gamma
+// with x_n = x * r, r = 1 / sqrt(mean(x^2) + eps). Inputs here are fp64 (so
+// finite differences can probe them); the bf16 forward above is the same
+// function of the same values.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct GradJob {
+  size_t seg;
+  int head;
+  int64_t lo, hi;  // rows of the sample (query rows or key rows), relative to its start
+};
+
+}  // namespace
+
+int oracle_attn_grad(const double* q, const double* k, const double* v, const double* gq_text,
+                     const double* gq_img, const double* gk_text, const double* gk_img,
+                     const double* dout, int n, const int32_t* n_text, const int32_t* grid_h,
+                     const int32_t* grid_w, const int32_t* frames, int heads, int d, double eps,
+                     int frame_dims, double scale, double* out, double* dq, double* dk, double* dv,
+                     double* dgamma, int n_threads) {
+  std::vector<Segment> segs;
+  int64_t total = 0;
+  if (!make_segments(n, n_text, grid_h, grid_w, frames, segs, total)) return -1;
+  if (heads < 1 || d < 4 || d % 4 != 0 || !valid_frame_dims(d, frame_dims)) return -1;
+  if (dout && (!dq || !dk || !dv || !dgamma)) return -1;
+  const size_t rows = static_cast<size_t>(total) * heads;
+
+  // Per (token, head) of q and k: r, x_n and the rotated x_hat.
+  std::vector<double> rq(rows), rk(rows), qn(rows * d), kn(rows * d), qh(rows * d), kh(rows * d);
+  std::vector<int64_t> pf(total), pr(total), pc(total);
+  std::vector<char> txt(total);
+  for (int64_t t = 0; t < total; ++t) {
+    bool is_text;
+    token_position(segs[segment_of(segs, t)], t, is_text, pf[t], pr[t], pc[t]);
+    txt[t] = is_text;
+    for (int h = 0; h < heads; ++h) {
+      const size_t row = static_cast<size_t>(t) * heads + h;
+      for (int which = 0; which < 2; ++which) {
+        const double* x = (which == 0 ? q : k) + row * d;
+        const double* g = which == 0 ? (is_text ? gq_text : gq_img) : (is_text ? gk_text : gk_img);
+        double sum_sq = 0.0;
+        for (int m = 0; m < d; ++m) sum_sq += x[m] * x[m];
+        const double r = 1.0 / std::sqrt(sum_sq / d + eps);
+        double* xn = (which == 0 ? qn : kn).data() + row * d;
+        double* xh = (which == 0 ? qh : kh).data() + row * d;
+        for (int m = 0; m < d; ++m) {
+          xn[m] = x[m] * r;
+          xh[m] = xn[m] * g[m];
+        }
+        if (!is_text) rotate_pairs(xh, d, frame_dims, pf[t], pr[t], pc[t], 1.0);
+        (which == 0 ? rq : rk)[row] = r;
+      }
+    }
+  }
+
+  auto score = [&](size_t row_q, size_t row_k) {
+    double dot = 0.0;
+    for (int m = 0; m < d; ++m) dot += qh[row_q * d + m] * kh[row_k * d + m];
+    return dot * scale;
+  };
+  auto run_jobs = [&](const std::vector<GradJob>& jobs, auto&& body) {
+    std::atomic<size_t> next{0};
+    auto worker = [&]() {
+      for (;;) {
+        size_t ji = next.fetch_add(1);
+        if (ji >= jobs.size()) break;
+        body(jobs[ji]);
+      }
+    };
+    int nt = std::min<int>(resolve_threads(n_threads), std::max<size_t>(jobs.size(), 1));
+    std::vector<std::thread> pool;
+    for (int i = 1; i < nt; ++i) pool.emplace_back(worker);
+    worker();
+    for (auto& th : pool) th.join();
+  };
+  std::vector<GradJob> jobs;
+  for (size_t si = 0; si < segs.size(); ++si)
+    for (int h = 0; h < heads; ++h)
+      for (int64_t lo = 0; lo < segs[si].len; lo += 64)
+        jobs.push_back({si, h, lo, std::min<int64_t>(segs[si].len, lo + 64)});
+
+  // Pass 1, per query row: M_t, Z_t, the output and (with a gradient) D_t.
+  std::vector<double> M(rows), Z(rows), D(rows, 0.0), o(rows * d);
+  run_jobs(jobs, [&](const GradJob& jb) {
+    const Segment& s = segs[jb.seg];
+    std::vector<double> sc(static_cast<size_t>(s.len));
+    for (int64_t i = jb.lo; i < jb.hi; ++i) {
+      const size_t rt = static_cast<size_t>(s.start + i) * heads + jb.head;
+      double mx = -std::numeric_limits<double>::infinity();
+      for (int64_t u = 0; u < s.len; ++u) {
+        sc[u] = score(rt, static_cast<size_t>(s.start + u) * heads + jb.head);
+        mx = std::max(mx, sc[u]);
+      }
+      double z = 0.0;
+      for (int64_t u = 0; u < s.len; ++u) z += std::exp(sc[u] - mx);
+      M[rt] = mx;
+      Z[rt] = z;
+      double* ot = &o[rt * d];
+      for (int m = 0; m < d; ++m) ot[m] = 0.0;
+      double dsum = 0.0;
+      for (int64_t u = 0; u < s.len; ++u) {
+        const size_t ru = static_cast<size_t>(s.start + u) * heads + jb.head;
+        const double p = std::exp(sc[u] - mx) / z;
+        for (int m = 0; m < d; ++m) ot[m] += p * v[ru * d + m];
+        if (dout) {
+          double dp = 0.0;
+          for (int m = 0; m < d; ++m) dp += dout[rt * d + m] * v[ru * d + m];
+          dsum += p * dp;
+        }
+      }
+      D[rt] = dsum;
+    }
+  });
+  if (out) std::copy(o.begin(), o.end(), out);
+  if (!dout) return 0;
+
+  // P_tu and dS_tu from the stored row statistics.
+  auto p_ds = [&](size_t rt, size_t ru, double& p, double& ds) {
+    p = std::exp(score(rt, ru) - M[rt]) / Z[rt];
+    double dp = 0.0;
+    for (int m = 0; m < d; ++m) dp += dout[rt * d + m] * v[ru * d + m];
+    ds = p * (dp - D[rt]);
+  };
+  // Pass 2, per query row: dq_hat.  Pass 3, per key row: dk_hat and dv.
+  std::vector<double> dqh(rows * d, 0.0), dkh(rows * d, 0.0);
+  run_jobs(jobs, [&](const GradJob& jb) {
+    const Segment& s = segs[jb.seg];
+    for (int64_t i = jb.lo; i < jb.hi; ++i) {
+      const size_t rt = static_cast<size_t>(s.start + i) * heads + jb.head;
+      double* acc = &dqh[rt * d];
+      for (int64_t u = 0; u < s.len; ++u) {
+        const size_t ru = static_cast<size_t>(s.start + u) * heads + jb.head;
+        double p, ds;
+        p_ds(rt, ru, p, ds);
+        for (int m = 0; m < d; ++m) acc[m] += scale * ds * kh[ru * d + m];
+      }
+    }
+  });
+  run_jobs(jobs, [&](const GradJob& jb) {
+    const Segment& s = segs[jb.seg];
+    for (int64_t i = jb.lo; i < jb.hi; ++i) {
+      const size_t ru = static_cast<size_t>(s.start + i) * heads + jb.head;
+      double* acc_k = &dkh[ru * d];
+      double* acc_v = dv + ru * d;
+      for (int m = 0; m < d; ++m) acc_v[m] = 0.0;
+      for (int64_t t = 0; t < s.len; ++t) {
+        const size_t rt = static_cast<size_t>(s.start + t) * heads + jb.head;
+        double p, ds;
+        p_ds(rt, ru, p, ds);
+        for (int m = 0; m < d; ++m) {
+          acc_k[m] += scale * ds * qh[rt * d + m];
+          acc_v[m] += p * dout[rt * d + m];
+        }
+      }
+    }
+  });
+
+  // Back through the rotation and the norm; gammas summed in token order.
+  for (int i = 0; i < 4 * d; ++i) dgamma[i] = 0.0;
+  std::vector<double> dy(d);
+  for (int64_t t = 0; t < total; ++t) {
+    for (int h = 0; h < heads; ++h) {
+      const size_t row = static_cast<size_t>(t) * heads + h;
+      for (int which = 0; which < 2; ++which) {
+        const double* dxh = (which == 0 ? dqh : dkh).data() + row * d;
+        const double* xn = (which == 0 ? qn : kn).data() + row * d;
+        const double* g = which == 0 ? (txt[t] ? gq_text : gq_img) : (txt[t] ? gk_text : gk_img);
+        const double r = (which == 0 ? rq : rk)[row];
+        double* dg = dgamma + (2 * which + (txt[t] ? 0 : 1)) * d;
+        double* dx = (which == 0 ? dq : dk) + row * d;
+        for (int m = 0; m < d; ++m) dy[m] = dxh[m];
+        if (!txt[t]) rotate_pairs(dy.data(), d, frame_dims, pf[t], pr[t], pc[t], -1.0);
+        double dot = 0.0;
+        for (int m = 0; m < d; ++m) {
+          dg[m] += dy[m] * xn[m];
+          dot += xn[m] * (dy[m] * g[m]);
+        }
+        for (int m = 0; m < d; ++m) dx[m] = r * (dy[m] * g[m] - xn[m] * dot / d);
       }
     }
   }
