@@ -202,8 +202,10 @@ extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_d
   prm.segs = segs_dev;
   prm.work = work_dev;
   prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
   prm.n_work = n_work;
   prm.heads = heads;
+  prm.total_tokens = total_tokens;
   prm.scale_log2 = scale * 1.4426950408889634f;
 
   // Persistent: one CTA per SM (or fewer if there are fewer items).

@@ -109,8 +109,10 @@ struct AttnParams {
   const mf_segment* segs;
   const mf_work_item* work;
   __nv_bfloat16* out;
+  float* lse;        // optional [heads, total_tokens]: natural-log softmax normaliser per row
   int n_work;
   int heads;
+  int total_tokens;
   float scale_log2;  // softmax scale * log2(e)
 };
 
@@ -520,6 +522,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int q_row = it.q0 + t * kSubM + row;
       const bool store = row_in;
       const float inv_l = 1.0f / l;
+      // log of the row's softmax normaliser, sum_u exp(s_u * scale), for the
+      // backward pass: m and l are in the exp2 domain of s * scale * log2(e).
+      if (p.lse && store)
+        p.lse[static_cast<size_t>(it.head) * p.total_tokens + q_row] =
+            (m + log2f(l)) * 0.6931471805599453f;
       uint4* dst = reinterpret_cast<uint4*>(p.out) +
                    (static_cast<size_t>(q_row) * p.heads + it.head) * (D / 8);
 #pragma unroll 1
