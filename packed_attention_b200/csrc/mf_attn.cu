@@ -172,11 +172,14 @@ extern "C" mf_status mf_qk_prologue(const void* q, const void* k, const float* g
                            workspace_bytes, stream);
 }
 
-extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_dev,
-                                         int32_t n_samples, const mf_work_item* work_dev,
-                                         int32_t n_work, int32_t total_tokens, int32_t heads,
-                                         int32_t head_dim, float softmax_scale, void* out,
-                                         void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+// Stage 2 with an optional per-row log-normaliser output (lse, [heads, T]).
+mf_status packed_attention_impl(const void* v, const mf_segment* segs_dev, int32_t n_samples,
+                                const mf_work_item* work_dev, int32_t n_work,
+                                int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                float softmax_scale, void* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream) {
   if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
   WorkspaceLayout w;
   if (!layout(total_tokens, heads, head_dim, &w) || n_samples < 1 || n_work < 1)
@@ -189,6 +192,13 @@ extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_d
   const size_t bytes = static_cast<size_t>(total_tokens) * heads * head_dim * 2;
   if (overlaps(out, bytes, v, bytes) || overlaps(out, bytes, workspace, w.total))
     return MF_ERR_INVALID_ARG;
+  if (lse) {
+    const size_t lse_bytes = static_cast<size_t>(total_tokens) * heads * 4;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return MF_ERR_ALIGNMENT;
+    if (overlaps(lse, lse_bytes, out, bytes) || overlaps(lse, lse_bytes, v, bytes) ||
+        overlaps(lse, lse_bytes, workspace, w.total))
+      return MF_ERR_INVALID_ARG;
+  }
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   CUtensorMap tq, tk, tv;
@@ -223,6 +233,18 @@ extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_d
         <<<grid, mf::kAttnThreads, mf::AttnConfig<64>::kSmemBytes, s>>>(tq, tk, tv, prm);
   }
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" mf_status mf_packed_attention(const void* v, const mf_segment* segs_dev,
+                                         int32_t n_samples, const mf_work_item* work_dev,
+                                         int32_t n_work, int32_t total_tokens, int32_t heads,
+                                         int32_t head_dim, float softmax_scale, void* out,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  return packed_attention_impl(v, segs_dev, n_samples, work_dev, n_work, total_tokens, heads,
+                               head_dim, softmax_scale, out, nullptr, workspace, workspace_bytes,
+                               stream);
 }
 
 extern "C" mf_status mf_joint_attn_fwd_3d(const void* q, const void* k, const void* v,
