@@ -295,6 +295,51 @@ def report_all(args):
             "prologue_gbs": 8 * T * H * d / (pro / 1e3) / 1e9,
             "rope_frame_dims": w.rope_frame_dims, "peaks": peak_src}), flush=True)
 
+    # Training: forward with the log-normaliser, then the backward (one call
+    # each). Backward FLOPs counted as 2.5x the forward's (five products of
+    # the forward's size: S recomputed, dP, dV, dK, dQ).
+    for key, w in [(1, WORKLOADS[1]), (2, WORKLOADS[2]), (3, WORKLOADS[3]), (4, WORKLOADS[4]),
+                   ("edit_1024sq_rope3d", EXTRA_WORKLOADS["edit_1024sq_rope3d"])]:
+        inp = make_inputs(w)
+        t, plan, ws, out, eps, fd = prepare(w, inp)
+        lse = torch.empty(w.heads, w.total_tokens, dtype=torch.float32, device=dev)
+        dout = torch.randn_like(out)
+        bws = torch.empty(pa.bwd_workspace_bytes(plan), dtype=torch.uint8, device=dev)
+        stream = torch.cuda.current_stream()
+
+        def fwd():
+            pa.joint_attention_fwd_lse(t["q"], t["k"], t["v"], t, plan, eps=eps, frame_dims=fd,
+                                       out=out, lse=lse, workspace=ws)
+
+        def bwd():
+            pa.joint_attention_bwd(t["q"], t["k"], t["v"], t, plan, out, lse, dout, eps=eps,
+                                   frame_dims=fd, workspace=bws)
+
+        for _ in range(max(3, args.warmup)):
+            fwd()
+            bwd()
+        torch.cuda.synchronize()
+        K = max(5, args.steps // 5)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        for e in evs:
+            e[0].record(stream)
+            fwd()
+            e[1].record(stream)
+            bwd()
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        if pa.device_error() != 0:
+            raise RuntimeError("kernel reported a device-side error")
+        f_ms = sorted(e[0].elapsed_time(e[1]) for e in evs)[K // 2]
+        b_ms = sorted(e[1].elapsed_time(e[2]) for e in evs)[K // 2]
+        print(json.dumps({
+            "workload": w.name, "config": key, "phase": "training", "gflop_forward": w.flops / 1e9,
+            "median_ms_forward_lse": f_ms, "median_ms_backward": b_ms,
+            "tflops_forward": w.flops / (f_ms / 1e3) / 1e12,
+            "tflops_backward": 2.5 * w.flops / (b_ms / 1e3) / 1e12,
+            "frac_sustained_peak_backward": 2.5 * w.flops / (b_ms / 1e3) / 1e12 / sustained,
+            "peaks": peak_src}), flush=True)
+
     for name, cp in CFG_PACKS.items():
         w = cp.packed()
         inp = make_inputs(w)

@@ -213,6 +213,56 @@ mf_status mf_joint_attn_fwd_3d(const void* q, const void* k, const void* v,
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Training: the forward with its per-row log-normaliser, and the backward.
+ * [The pages measure their fused-kernel speedup on training the NR-MMDiT:
+ *  video overview, 00:05:08; paper summary, "Training Infrastructure".]
+ *
+ * mf_joint_attn_fwd_lse -- mf_joint_attn_fwd_3d that also writes
+ *   lse     fp32 [heads, total_tokens] (head-major), device, 4-B aligned:
+ *           lse[h, t] = log(sum_u exp(scale * q_hat_t . k_hat_u)) over the
+ *           keys u of t's sample (natural log). The backward needs it.
+ *
+ * mf_bwd_workspace_bytes -- device workspace mf_joint_attn_bwd needs
+ *   (q_hat, k_hat, the row terms D = rowsum(dout * out), fp32 dq_hat and
+ *   dk_hat, and the per-block gamma-gradient partials). 0 for invalid sizes.
+ *
+ * mf_joint_attn_bwd -- gradients of the forward for dL/dout = dout:
+ *   inputs   q, k, v, the four gammas, the plan arrays, eps, frame_dims and
+ *            softmax_scale exactly as given to the forward; out (bf16
+ *            [T, H, d]) and lse as the forward wrote them; dout (bf16
+ *            [T, H, d], 16-B aligned).
+ *   outputs  dq, dk, dv (bf16 [T, H, d], 16-B aligned) and dgamma (fp32
+ *            [4, head_dim] in the order q_text, q_img, k_text, k_img: each
+ *            summed over all tokens and heads of its role and modality).
+ *            Outputs must not overlap the inputs, the workspace or one
+ *            another (MF_ERR_INVALID_ARG).
+ *   The chain rule through the attention (dS = P * (dP - D)), the rotation
+ *   (transposed) and the RMSNorm. Every result is deterministic: no atomics;
+ *   the gamma sums run in a fixed order. Asynchronous on `stream`.
+ *   Errors as for mf_joint_attn_fwd_3d; MF_ERR_WORKSPACE when
+ *   workspace_bytes < mf_bwd_workspace_bytes(...).
+ */
+mf_status mf_joint_attn_fwd_lse(const void* q, const void* k, const void* v,
+                                const float* g_q_text, const float* g_q_img,
+                                const float* g_k_text, const float* g_k_img,
+                                const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                                int32_t n_samples, const mf_work_item* work_dev, int32_t n_work,
+                                int32_t total_tokens, int32_t heads, int32_t head_dim, float eps,
+                                int32_t frame_dims, float softmax_scale, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+size_t mf_bwd_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim);
+
+mf_status mf_joint_attn_bwd(const void* q, const void* k, const void* v, const float* g_q_text,
+                            const float* g_q_img, const float* g_k_text, const float* g_k_img,
+                            const void* out, const void* dout, const float* lse,
+                            const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                            int32_t n_samples, const mf_work_item* work_dev, int32_t n_work,
+                            int32_t total_tokens, int32_t heads, int32_t head_dim, float eps,
+                            int32_t frame_dims, float softmax_scale, void* dq, void* dk, void* dv,
+                            float* dgamma, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * mf_joint_attn_fwd_static_scratch -- the same forward for callers that
  * cannot allocate device memory at all. The paper has no counterpart to this
  * entry point; it exists for how the library is called, not for the method.

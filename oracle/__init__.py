@@ -56,7 +56,7 @@ def _load():
                                               i32, dbl, i64, P, P, i32]
             lib.oracle_attn_grad.restype = i32
             lib.oracle_attn_grad.argtypes = [P, P, P, P, P, P, P, P, i32, P, P, P, P, i32, i32, dbl,
-                                             i32, dbl, P, P, P, P, P, i32]
+                                             i32, dbl, P, P, P, P, P, P, i32]
             lib.oracle_dense_attn.restype = i32
             lib.oracle_dense_attn.argtypes = [P, P, P, P, P, P, P, i32, P, P, P, P, i32, i32, dbl,
                                               i32, dbl, P]
@@ -155,7 +155,8 @@ def dense_attn(q, k, v, gammas, samples, eps=1e-6, scale=None, frame_dims=0):
 
 def attn_grad(q, k, v, gammas, samples, dout=None, eps=1e-6, scale=None, frame_dims=0,
               n_threads=0):
-    """Forward output and, given ``dout`` = dL/dout, the gradients, all fp64.
+    """Forward output, the per-row log-normaliser ``lse`` (``[T, H]``, natural
+    log of sum_u exp(s_tu)) and, given ``dout`` = dL/dout, the gradients, all fp64.
 
     q, k, v, dout: float64 ``[T, H, d]`` values (not bf16 bits); gammas: dict of
     the four ``[d]`` vectors. Returns a dict with ``out`` and, with ``dout``,
@@ -172,7 +173,8 @@ def attn_grad(q, k, v, gammas, samples, dout=None, eps=1e-6, scale=None, frame_d
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     out = np.empty((T, H, d), dtype=np.float64)
-    res = {"out": out}
+    lse = np.empty((T, H), dtype=np.float64)
+    res = {"out": out, "lse": lse}
     go = dq = dk = dv = dg = None
     if dout is not None:
         go = np.ascontiguousarray(dout, dtype=np.float64)
@@ -182,7 +184,8 @@ def attn_grad(q, k, v, gammas, samples, dout=None, eps=1e-6, scale=None, frame_d
         dg = np.empty((4, d), dtype=np.float64)
     rc = _load().oracle_attn_grad(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in g], _ptr(go), n,
                                   _ptr(nt), _ptr(gh), _ptr(gw), _ptr(fr), H, d, float(eps),
-                                  int(frame_dims), float(scale), _ptr(out), _ptr(dq), _ptr(dk),
+                                  int(frame_dims), float(scale), _ptr(out), _ptr(lse), _ptr(dq),
+                                  _ptr(dk),
                                   _ptr(dv), _ptr(dg), int(n_threads))
     if rc != 0:
         raise ValueError("oracle_attn_grad rejected its arguments")

@@ -435,8 +435,8 @@ int oracle_attn_grad(const double* q, const double* k, const double* v, const do
                      const double* gq_img, const double* gk_text, const double* gk_img,
                      const double* dout, int n, const int32_t* n_text, const int32_t* grid_h,
                      const int32_t* grid_w, const int32_t* frames, int heads, int d, double eps,
-                     int frame_dims, double scale, double* out, double* dq, double* dk, double* dv,
-                     double* dgamma, int n_threads) {
+                     int frame_dims, double scale, double* out, double* lse, double* dq,
+                     double* dk, double* dv, double* dgamma, int n_threads) {
   std::vector<Segment> segs;
   int64_t total = 0;
   if (!make_segments(n, n_text, grid_h, grid_w, frames, segs, total)) return -1;
@@ -531,6 +531,8 @@ int oracle_attn_grad(const double* q, const double* k, const double* v, const do
     }
   });
   if (out) std::copy(o.begin(), o.end(), out);
+  if (lse)  // log of the softmax normaliser: log sum_u exp(s_tu) = M_t + log Z_t, [T, heads]
+    for (size_t r = 0; r < rows; ++r) lse[r] = M[r] + std::log(Z[r]);
   if (!dout) return 0;
 
   // P_tu and dS_tu from the stored row statistics.

@@ -1,4 +1,5 @@
-"""B200-native packed joint text+image attention forward (Mage-Flow NR-MMDiT hot path).
+"""B200-native packed joint text+image attention (Mage-Flow NR-MMDiT hot path):
+forward, and the backward for training.
 
 The compute lives in ``libmfattn.so`` (hand-written sm_100a CUDA behind the C ABI
 in ``include/mf_attn.h``); this package marshals torch tensors into it.
@@ -9,12 +10,15 @@ from ._native import MfError, MF_TILE_M, MF_TILE_N, pack_plan, workspace_bytes  
 
 __all__ = ["MfError", "MF_TILE_M", "MF_TILE_N", "pack_plan", "workspace_bytes",
            "PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
-           "packed_attention", "workspace_views", "device_error"]
+           "packed_attention", "workspace_views", "device_error", "joint_attention_fwd_lse",
+           "joint_attention_bwd", "joint_attention_autograd", "bwd_workspace_bytes"]
 
 
 def __getattr__(name):
     if name in ("PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
-                "packed_attention", "workspace_views", "device_error", "GAMMA_NAMES"):
+                "packed_attention", "workspace_views", "device_error", "GAMMA_NAMES",
+                "joint_attention_fwd_lse", "joint_attention_bwd", "joint_attention_autograd",
+                "bwd_workspace_bytes", "JointAttentionFunction"):
         from . import api
         return getattr(api, name)
     raise AttributeError(name)

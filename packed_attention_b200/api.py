@@ -170,3 +170,90 @@ def joint_attention_host(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
 def device_error(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the kernels' error code."""
     return int(lib().mf_get_device_error(_stream_handle(stream)))
+
+
+# ------------------------------------------------------------- training ---
+
+def joint_attention_fwd_lse(q, k, v, gammas, plan: PackedPlan, eps: float = 1e-6,
+                            softmax_scale: float = 0.0, frame_dims: int = 0,
+                            out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                            workspace: torch.Tensor | None = None, stream=None):
+    """Forward that also returns the per-row natural log-normaliser
+    ``lse`` (fp32 ``[H, T]``) the backward needs. Returns ``(out, lse)``."""
+    _check_qkv(plan, q, k, v)
+    gs = _gammas(gammas, plan)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_qkv(plan, out)
+    if lse is None:
+        lse = torch.empty(plan.heads, plan.total_tokens, dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (plan.heads, plan.total_tokens) \
+            or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor of shape [heads, total_tokens]")
+    if workspace is None:
+        workspace = plan.new_workspace()
+    check("mf_joint_attn_fwd_lse", lib().mf_joint_attn_fwd_lse(
+        _ptr(q), _ptr(k), _ptr(v), *[_ptr(g) for g in gs], _ptr(plan.cu_seqlens),
+        _ptr(plan.segs), plan.n_samples, _ptr(plan.work), plan.n_work, plan.total_tokens,
+        plan.heads, plan.head_dim, float(eps), int(frame_dims), float(softmax_scale), _ptr(out),
+        _ptr(lse), _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    return out, lse
+
+
+def bwd_workspace_bytes(plan: PackedPlan) -> int:
+    return int(lib().mf_bwd_workspace_bytes(plan.total_tokens, plan.heads, plan.head_dim))
+
+
+def joint_attention_bwd(q, k, v, gammas, plan: PackedPlan, out, lse, dout, eps: float = 1e-6,
+                        softmax_scale: float = 0.0, frame_dims: int = 0,
+                        workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """Gradients of the forward for ``dL/dout = dout``: a dict with ``dq``,
+    ``dk``, ``dv`` (bf16 ``[T, H, d]``) and one fp32 ``[d]`` gradient per gamma
+    (keys ``g_q_text`` ...)."""
+    _check_qkv(plan, q, k, v, out, dout)
+    gs = _gammas(gammas, plan)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dgamma = torch.empty(4, plan.head_dim, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(plan), dtype=torch.uint8, device=q.device)
+    check("mf_joint_attn_bwd", lib().mf_joint_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), *[_ptr(g) for g in gs], _ptr(out), _ptr(dout), _ptr(lse),
+        _ptr(plan.cu_seqlens), _ptr(plan.segs), plan.n_samples, _ptr(plan.work), plan.n_work,
+        plan.total_tokens, plan.heads, plan.head_dim, float(eps), int(frame_dims),
+        float(softmax_scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgamma), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream)))
+    res = {"dq": dq, "dk": dk, "dv": dv}
+    res.update({n: dgamma[i] for i, n in enumerate(GAMMA_NAMES)})
+    return res
+
+
+class JointAttentionFunction(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run in libmfattn's kernels.
+
+    ``joint_attention_autograd(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img,
+    plan, eps, softmax_scale, frame_dims)``; gradients flow to q, k, v and the
+    four gammas."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, plan, eps, softmax_scale,
+                frame_dims):
+        gammas = dict(zip(GAMMA_NAMES, (g_q_text, g_q_img, g_k_text, g_k_img)))
+        out, lse = joint_attention_fwd_lse(q, k, v, gammas, plan, eps, softmax_scale, frame_dims)
+        ctx.save_for_backward(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, out, lse)
+        ctx.plan, ctx.eps, ctx.scale, ctx.frame_dims = plan, eps, softmax_scale, frame_dims
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, gqt, gqi, gkt, gki, out, lse = ctx.saved_tensors
+        gammas = dict(zip(GAMMA_NAMES, (gqt, gqi, gkt, gki)))
+        g = joint_attention_bwd(q, k, v, gammas, ctx.plan, out, lse,
+                                dout.to(torch.bfloat16).contiguous(), ctx.eps, ctx.scale,
+                                ctx.frame_dims)
+        return (g["dq"], g["dk"], g["dv"], *[g[n] for n in GAMMA_NAMES], None, None, None, None)
+
+
+def joint_attention_autograd(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, plan: PackedPlan,
+                             eps: float = 1e-6, softmax_scale: float = 0.0, frame_dims: int = 0):
+    return JointAttentionFunction.apply(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, plan, eps,
+                                        softmax_scale, frame_dims)

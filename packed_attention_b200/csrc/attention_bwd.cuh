@@ -1,0 +1,638 @@
+// Backward of the packed joint attention, for training.
+//
+// [Mage-Flow video overview, 00:05:08, and paper summary, "Training
+//  Infrastructure": the fused-kernel speedup is a training speedup. The
+//  backward here is the chain rule through the forward of this library.]
+//
+// With dO = dL/dout, the forward's bf16 output `out` and its per-row natural
+// log-normaliser lse (written by the forward), for query t and key u of one
+// sample and head, s_tu = scale * q_hat_t . k_hat_u:
+//   D_t       = dO_t . out_t                                   bwd_delta_kernel
+//   P_tu      = exp(s_tu - lse_t)                              (recomputed)
+//   dS_tu     = P_tu * (dO_t . v_u - D_t)
+//   dv_u      = sum_t P_tu dO_t                                attn_bwd_dkdv_kernel
+//   dk_hat_u  = scale * sum_t dS_tu q_hat_t                    attn_bwd_dkdv_kernel
+//   dq_hat_t  = scale * sum_u dS_tu k_hat_u                    attn_bwd_dq_kernel
+// then back through the rotation (transposed) and the RMSNorm, with the four
+// gamma gradients summed over tokens and heads    qk_prologue_bwd_kernel,
+//                                                  dgamma_reduce_kernel
+//
+// The two attention kernels are persistent tcgen05 kernels built like the
+// forward: TMA loads into 128-byte-swizzled shared tiles, MMAs issued by one
+// thread with fp32 accumulators in TMEM, eight softmax warps (a TMEM lane
+// quarter each, two warps per quarter splitting the 128 columns), bounded
+// mbarrier waits throughout. A work item of the forward's list (256 rows of
+// one head of one sample) is done as two passes of 128 rows.
+//
+// dK/dV kernel, per pass: 128 key rows; K_hat and V stay in shared memory and
+// every query step j brings Q_hat_j and dO_j (two rings). TMEM columns:
+//   S^T = K_hat Q_hat_j^T [0,128)   P^T (bf16) over its columns [0,32) and [64,96)
+//   dP^T = V dO_j^T     [128,256)   dS^T (bf16) over [128,160) and [192,224)
+//   dV accumulator      [256,256+d)
+//   dK accumulator      [384,384+d)
+// MMA order per step: dV_j, S^T_{j+1}, dK_j, dP^T_{j+1}. The softmax computes
+// P^T_{j+1} while the tensor core runs dK_j and dP^T_{j+1}, and dS^T_{j+1}
+// while it runs dV_{j+1} and S^T_{j+2}. MMAs of one thread execute in issue
+// order, so S^T_{j+1} overwrites P^T_j only after dV_j has read it (and
+// dP^T_{j+1} overwrites dS^T_j only after dK_j).
+//
+// dQ kernel, per pass: 128 query rows; Q_hat and dO stay, every key step
+// brings K_hat_j and V_j. TMEM: S [0,128), dP [128,256) with dS (bf16) written
+// over its columns [128,160) and [192,224), dQ accumulator [256,256+d). S_{j+1}
+// is issued as soon as every softmax warp has loaded S_j into registers;
+// order per step: S_{j+1}, dQ_j, dP_{j+1}.
+#pragma once
+
+#include "packed_attention.cuh"
+
+namespace mf {
+
+constexpr int kBwdThreads = 320;
+constexpr int kBwdProducerWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// kRingX: the operand held longest (Q_hat in dK/dV, K_hat in dQ);
+// kRingY: the one released after its first MMA (dO in dK/dV, V in dQ).
+template <int D, bool kDq>
+struct BwdConfig {
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kTileBytes = kSubM * D * 2;
+  static constexpr int kRingX = (kDq || D == 64) ? 3 : 2;
+  static constexpr int kRingY = 2;
+  static constexpr int kSmemBytes = kTileBytes * (2 + kRingX + kRingY) + 1024;
+};
+
+struct BwdParams {
+  const mf_segment* segs;
+  const mf_work_item* work;
+  const float* lse;       // [heads, total_tokens], natural log
+  const float* delta;     // [heads, total_tokens]
+  float* dhat;            // fp32 [total_tokens, heads, D]: dk_hat or dq_hat
+  __nv_bfloat16* dv;      // bf16 [total_tokens, heads, D] (dK/dV kernel)
+  int n_work;
+  int heads;
+  int total_tokens;
+  float scale;            // softmax scale
+  float scale_log2;       // scale * log2(e)
+};
+
+struct BwdCtl {
+  uint64_t fix_full, fix_empty;
+  uint64_t x_full[3], x_empty[3];
+  uint64_t y_full[2], y_empty[2];
+  uint64_t s_full, s_free, dp_full;
+  uint64_t p_ready, ds_ready;
+  uint64_t acc_ready, acc_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+// D (+)= A (TMEM, bf16: 128 lanes x 128 K, K 0..63 in columns [0,32) and
+// K 64..127 in [64,96)) * B (shared, MN-major [K = 128 rows][N = D]).
+template <int D>
+__device__ __forceinline__ void issue_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             bool accumulate) {
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts(d_tmem, a_tmem + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+           b_desc + static_cast<uint64_t>(kk * (2048 >> 4)), kIdesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int D, bool kDq>
+__device__ __forceinline__ void bwd_init(BwdCtl& ctl, int warp) {
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl.fix_full, 1);
+    mbar_init(&ctl.fix_empty, 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&ctl.x_full[s], 1);
+      mbar_init(&ctl.x_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl.y_full[s], 1);
+      mbar_init(&ctl.y_empty[s], 1);
+    }
+    mbar_init(&ctl.s_full, 1);
+    mbar_init(&ctl.s_free, 8);
+    mbar_init(&ctl.dp_full, 1);
+    mbar_init(&ctl.p_ready, 8);
+    mbar_init(&ctl.ds_ready, 8);
+    mbar_init(&ctl.acc_ready, 1);
+    mbar_init(&ctl.acc_empty, 8);
+    mbar_init(&ctl.drain, 1);
+    ctl.abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(&ctl.tmem_base, kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+}
+
+__device__ __forceinline__ void bwd_teardown(uint32_t tmem, int warp) {
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Producer for both kernels: per pass, the two fixed tiles (rows r0 of
+// fix_a / fix_b), then per step j the ring tiles (rows seg_start + 128 j of
+// ring_x / ring_y).
+template <int D, bool kDq>
+__device__ __forceinline__ void bwd_producer(const BwdParams& p, BwdCtl& ctl, uint8_t* sFix,
+                                             uint8_t* sX, uint8_t* sY, const CUtensorMap* fix_a,
+                                             const CUtensorMap* fix_b, const CUtensorMap* ring_x,
+                                             const CUtensorMap* ring_y,
+                                             volatile int32_t* abort_flag) {
+  using Cfg = BwdConfig<D, kDq>;
+  constexpr int NX = Cfg::kRingX, NY = Cfg::kRingY, kTile = Cfg::kTileBytes;
+  const int stride = static_cast<int>(gridDim.x);
+  int pc = 0, gx = 0, gy = 0;
+  bool ok = true;
+  for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+    const ItemInfo it = load_item(p.segs, p.work, idx);
+    const int passes = it.b_valid ? 2 : 1;
+    for (int t = 0; t < passes && ok; ++t) {
+      const int r0 = it.q0 + t * kSubM;
+      if (!wait_bar(&ctl.fix_empty, (pc & 1) ^ 1, abort_flag)) { ok = false; break; }
+      mbar_arrive_expect_tx(&ctl.fix_full, 2 * kTile);
+#pragma unroll
+      for (int b = 0; b < Cfg::kBoxes; ++b) {
+        tma_load_3d(sFix + b * kBoxBytes, fix_a, &ctl.fix_full, 64 * b, it.head, r0);
+        tma_load_3d(sFix + kTile + b * kBoxBytes, fix_b, &ctl.fix_full, 64 * b, it.head, r0);
+      }
+      ++pc;
+      for (int j = 0; j < it.n_kv && ok; ++j) {
+        const int c = it.seg_start + j * kBlockN;
+        {
+          const int st = gx % NX;
+          if (!wait_bar(&ctl.x_empty[st], ((gx / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&ctl.x_full[st], kTile);
+#pragma unroll
+          for (int b = 0; b < Cfg::kBoxes; ++b)
+            tma_load_3d(sX + st * kTile + b * kBoxBytes, ring_x, &ctl.x_full[st], 64 * b, it.head, c);
+          ++gx;
+        }
+        {
+          const int st = gy % NY;
+          if (!wait_bar(&ctl.y_empty[st], ((gy / NY) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&ctl.y_full[st], kTile);
+#pragma unroll
+          for (int b = 0; b < Cfg::kBoxes; ++b)
+            tma_load_3d(sY + st * kTile + b * kBoxBytes, ring_y, &ctl.y_full[st], 64 * b, it.head, c);
+          ++gy;
+        }
+      }
+    }
+  }
+  if (!ok) {
+    // Let every copy already issued land before the CTA can exit.
+    if (pc > 0) wait_slow(&ctl.fix_full, (pc - 1) & 1, nullptr, kDrainLimitNs);
+    for (int i = gx - NX > 0 ? gx - NX : 0; i < gx; ++i)
+      wait_slow(&ctl.x_full[i % NX], (i / NX) & 1, nullptr, kDrainLimitNs);
+    for (int i = gy - NY > 0 ? gy - NY : 0; i < gy; ++i)
+      wait_slow(&ctl.y_full[i % NY], (i / NY) & 1, nullptr, kDrainLimitNs);
+  }
+}
+
+// Passes and steps this CTA will run (for releasing only refilled slots).
+__device__ __forceinline__ void bwd_counts(const BwdParams& p, int& passes, int& steps) {
+  passes = steps = 0;
+  for (int idx = blockIdx.x; idx < p.n_work; idx += static_cast<int>(gridDim.x)) {
+    const ItemInfo it = load_item(p.segs, p.work, idx);
+    const int np = it.b_valid ? 2 : 1;
+    passes += np;
+    steps += np * it.n_kv;
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV ---
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                         const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v,
+                         const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
+  using Cfg = BwdConfig<D, false>;
+  constexpr int NX = Cfg::kRingX, NY = Cfg::kRingY, kTile = Cfg::kTileBytes;
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ BwdCtl ctl;
+  __shared__ __align__(16) float s_stat[8][2][64];  // per softmax warp: lse (log2) and D
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;              // fixed: K_hat then V
+  uint8_t* sV = smem + kTile;
+  uint8_t* sX = smem + 2 * kTile;  // ring of Q_hat
+  uint8_t* sY = sX + NX * kTile;   // ring of dO
+  volatile int32_t* abort_flag = &ctl.abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (warp == kBwdProducerWarp && lane == 0) {
+    prefetch_tmap(&tmap_q);
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_v);
+    prefetch_tmap(&tmap_do);
+  }
+  bwd_init<D, false>(ctl, warp);
+  const uint32_t tmem = ctl.tmem_base;
+  const int stride = static_cast<int>(gridDim.x);
+
+  if (warp == kBwdProducerWarp) {
+    if (lane == 0)
+      bwd_producer<D, false>(p, ctl, sK, sX, sY, &tmap_k, &tmap_v, &tmap_q, &tmap_do, abort_flag);
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0) {
+      const uint64_t k_desc = smem_desc_sw128(smem_addr(sK), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_addr(sV), 16, 1024);
+      const uint64_t x_k = smem_desc_sw128(smem_addr(sX), 16, 1024);          // Q_hat as B of S^T
+      const uint64_t x_mn = smem_desc_sw128(smem_addr(sX), kBoxBytes, 1024);  // Q_hat as B of dK
+      const uint64_t y_k = smem_desc_sw128(smem_addr(sY), 16, 1024);          // dO as B of dP^T
+      const uint64_t y_mn = smem_desc_sw128(smem_addr(sY), kBoxBytes, 1024);  // dO as B of dV
+      constexpr uint64_t kStep = static_cast<uint64_t>(kTile >> 4);
+      int total_passes, total_steps;
+      bwd_counts(p, total_passes, total_steps);
+      int pc = 0, g = 0;
+      uint32_t nph = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+        const ItemInfo it = load_item(p.segs, p.work, idx);
+        const int passes = it.b_valid ? 2 : 1;
+        for (int t = 0; t < passes && ok; ++t) {
+          const int n = it.n_kv;
+          if (!wait_bar(&ctl.fix_full, pc & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          if (!wait_bar(&ctl.x_full[g % NX], (g / NX) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          issue_qk<D>(tmem + kColS, k_desc, x_k + (g % NX) * kStep);
+          mma_commit(&ctl.s_full);
+          if (!wait_bar(&ctl.y_full[g % NY], (g / NY) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          issue_qk<D>(tmem + kColDP, v_desc, y_k + (g % NY) * kStep);
+          mma_commit(&ctl.dp_full);
+          for (int j = 0; j < n && ok; ++j) {
+            const int gj = g + j, gn = gj + 1;
+            const bool more = j + 1 < n;
+            if (!wait_bar(&ctl.p_ready, nph & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after_sync();
+            if (j == 0 && pc > 0) {
+              // the previous pass's accumulators have been read out
+              if (!wait_bar(&ctl.acc_empty, (pc - 1) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+            }
+            issue_tmem_a<D>(tmem + kColDV, tmem + kColS, y_mn + (gj % NY) * kStep, j > 0);
+            if (gj + NY < total_steps) mma_commit(&ctl.y_empty[gj % NY]);
+            if (more) {
+              if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_qk<D>(tmem + kColS, k_desc, x_k + (gn % NX) * kStep);
+              mma_commit(&ctl.s_full);
+            }
+            if (!wait_bar(&ctl.ds_ready, nph & 1, abort_flag)) { ok = false; break; }
+            ++nph;
+            tc_fence_after_sync();
+            issue_tmem_a<D>(tmem + kColDK, tmem + kColDP, x_mn + (gj % NX) * kStep, j > 0);
+            if (gj + NX < total_steps) mma_commit(&ctl.x_empty[gj % NX]);
+            if (more) {
+              if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_qk<D>(tmem + kColDP, v_desc, y_k + (gn % NY) * kStep);
+              mma_commit(&ctl.dp_full);
+            }
+          }
+          if (!ok) break;
+          if (pc + 1 < total_passes) mma_commit(&ctl.fix_empty);
+          mma_commit(&ctl.acc_ready);
+          g += n;
+          ++pc;
+        }
+      }
+      if (!ok) {
+        mma_commit(&ctl.drain);
+        wait_slow(&ctl.drain, 0, nullptr, kDrainLimitNs);
+      }
+    }
+  } else {
+    // ------------------------------------------- softmax and epilogue ---
+    const int g4 = warp & 3, h = warp >> 2;  // TMEM lane quarter, column half
+    const int row = g4 * 32 + lane;          // key row of the pass
+    const uint32_t lane_off = static_cast<uint32_t>(g4 * 32) << 16;
+    const float sl2 = p.scale_log2;
+    float* st_l = s_stat[warp][0];
+    float* st_d = s_stat[warp][1];
+    uint32_t ns = 0, nd = 0;
+    int pc = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+      const ItemInfo it = load_item(p.segs, p.work, idx);
+      const int passes = it.b_valid ? 2 : 1;
+      const int seg_end = it.seg_start + it.seg_len;
+      const size_t stat0 = static_cast<size_t>(it.head) * p.total_tokens;
+      for (int t = 0; t < passes && ok; ++t, ++pc) {
+        const int r0 = it.q0 + t * kSubM;
+        const bool row_in = r0 + row < seg_end;
+        for (int j = 0; j < it.n_kv; ++j) {
+          // lse (log2 units) and D of this warp's 64 queries; queries past
+          // the sample end get lse = +inf, hence P = 0 and dS = 0.
+          {
+            const int qa = it.seg_start + j * kBlockN + 64 * h + lane, qb = qa + 32;
+            const float la = qa < seg_end ? __ldg(p.lse + stat0 + qa) * kLog2e : INFINITY;
+            const float lb = qb < seg_end ? __ldg(p.lse + stat0 + qb) * kLog2e : INFINITY;
+            const float da = qa < seg_end ? __ldg(p.delta + stat0 + qa) : 0.0f;
+            const float db = qb < seg_end ? __ldg(p.delta + stat0 + qb) : 0.0f;
+            __syncwarp();
+            st_l[lane] = la;
+            st_l[lane + 32] = lb;
+            st_d[lane] = da;
+            st_d[lane + 32] = db;
+            __syncwarp();
+          }
+          if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
+          ++ns;
+          tc_fence_after_sync();
+          float pv[64];
+          {
+            uint32_t sr[64];
+            tmem_ld64_sync(tmem + lane_off + kColS + 64 * h, sr);
+            uint32_t pk[32];
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) {
+              const float4 l = reinterpret_cast<const float4*>(st_l)[c4];
+              pv[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), sl2, -l.x));
+              pv[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l.y));
+              pv[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l.z));
+              pv[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l.w));
+              pk[2 * c4] = pack_bf16x2(pv[4 * c4 + 0], pv[4 * c4 + 1]);
+              pk[2 * c4 + 1] = pack_bf16x2(pv[4 * c4 + 2], pv[4 * c4 + 3]);
+            }
+            tmem_st32_sync(tmem + lane_off + kColS + 64 * h, pk);
+          }
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.p_ready);
+          if (!warp_wait_bar(&ctl.dp_full, nd & 1, abort_flag)) { ok = false; break; }
+          ++nd;
+          tc_fence_after_sync();
+          {
+            uint32_t dr[64];
+            tmem_ld64_sync(tmem + lane_off + kColDP + 64 * h, dr);
+            uint32_t pk[32];
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) {
+              const float4 dd = reinterpret_cast<const float4*>(st_d)[c4];
+              const float d0 = pv[4 * c4 + 0] * (__uint_as_float(dr[4 * c4 + 0]) - dd.x);
+              const float d1 = pv[4 * c4 + 1] * (__uint_as_float(dr[4 * c4 + 1]) - dd.y);
+              const float d2 = pv[4 * c4 + 2] * (__uint_as_float(dr[4 * c4 + 2]) - dd.z);
+              const float d3 = pv[4 * c4 + 3] * (__uint_as_float(dr[4 * c4 + 3]) - dd.w);
+              pk[2 * c4] = pack_bf16x2(d0, d1);
+              pk[2 * c4 + 1] = pack_bf16x2(d2, d3);
+            }
+            tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
+          }
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.ds_ready);
+        }
+        if (!ok) break;
+        // ---- epilogue: dv (bf16) and dk_hat = scale * acc (fp32) rows ----
+        if (!warp_wait_bar(&ctl.acc_ready, pc & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after_sync();
+        const size_t orow = (static_cast<size_t>(r0 + row) * p.heads + it.head) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          const int col = h * (D / 2) + 32 * c;
+          uint32_t r[32];
+          tmem_ld32_sync(tmem + lane_off + kColDV + col, r);
+          if (row_in) {
+            uint4* dst = reinterpret_cast<uint4*>(p.dv + orow + col);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v4 + 0]), __uint_as_float(r[8 * v4 + 1]));
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]), __uint_as_float(r[8 * v4 + 3]));
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5]));
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7]));
+              dst[v4] = o;
+            }
+          }
+          tmem_ld32_sync(tmem + lane_off + kColDK + col, r);
+          if (row_in) {
+            float4* dst = reinterpret_cast<float4*>(p.dhat + orow + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(r[4 * v + 0]) * p.scale,
+                                   __uint_as_float(r[4 * v + 1]) * p.scale,
+                                   __uint_as_float(r[4 * v + 2]) * p.scale,
+                                   __uint_as_float(r[4 * v + 3]) * p.scale);
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.acc_empty);
+      }
+    }
+  }
+  bwd_teardown(tmem, warp);
+}
+
+// -------------------------------------------------------------------- dQ ---
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                       const __grid_constant__ CUtensorMap tmap_k,
+                       const __grid_constant__ CUtensorMap tmap_v,
+                       const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
+  using Cfg = BwdConfig<D, true>;
+  constexpr int NX = Cfg::kRingX, NY = Cfg::kRingY, kTile = Cfg::kTileBytes;
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ BwdCtl ctl;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;              // fixed: Q_hat then dO
+  uint8_t* sO = smem + kTile;
+  uint8_t* sX = smem + 2 * kTile;  // ring of K_hat
+  uint8_t* sY = sX + NX * kTile;   // ring of V
+  volatile int32_t* abort_flag = &ctl.abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (warp == kBwdProducerWarp && lane == 0) {
+    prefetch_tmap(&tmap_q);
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_v);
+    prefetch_tmap(&tmap_do);
+  }
+  bwd_init<D, true>(ctl, warp);
+  const uint32_t tmem = ctl.tmem_base;
+  const int stride = static_cast<int>(gridDim.x);
+
+  if (warp == kBwdProducerWarp) {
+    if (lane == 0)
+      bwd_producer<D, true>(p, ctl, sQ, sX, sY, &tmap_q, &tmap_do, &tmap_k, &tmap_v, abort_flag);
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0) {
+      const uint64_t q_desc = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+      const uint64_t o_desc = smem_desc_sw128(smem_addr(sO), 16, 1024);
+      const uint64_t x_k = smem_desc_sw128(smem_addr(sX), 16, 1024);          // K_hat as B of S
+      const uint64_t x_mn = smem_desc_sw128(smem_addr(sX), kBoxBytes, 1024);  // K_hat as B of dQ
+      const uint64_t y_k = smem_desc_sw128(smem_addr(sY), 16, 1024);          // V as B of dP
+      constexpr uint64_t kStep = static_cast<uint64_t>(kTile >> 4);
+      int total_passes, total_steps;
+      bwd_counts(p, total_passes, total_steps);
+      int pc = 0, g = 0;
+      uint32_t nph = 0, nsf = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+        const ItemInfo it = load_item(p.segs, p.work, idx);
+        const int passes = it.b_valid ? 2 : 1;
+        for (int t = 0; t < passes && ok; ++t) {
+          const int n = it.n_kv;
+          if (!wait_bar(&ctl.fix_full, pc & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          if (!wait_bar(&ctl.x_full[g % NX], (g / NX) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          issue_qk<D>(tmem + kColS, q_desc, x_k + (g % NX) * kStep);
+          mma_commit(&ctl.s_full);
+          if (!wait_bar(&ctl.y_full[g % NY], (g / NY) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          issue_qk<D>(tmem + kColDP, o_desc, y_k + (g % NY) * kStep);
+          mma_commit(&ctl.dp_full);
+          if (g + NY < total_steps) mma_commit(&ctl.y_empty[g % NY]);
+          for (int j = 0; j < n && ok; ++j) {
+            const int gj = g + j, gn = gj + 1;
+            const bool more = j + 1 < n;
+            if (more) {
+              // S_{j+1} as soon as every softmax warp holds S_j in registers
+              if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
+              ++nsf;
+              if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_qk<D>(tmem + kColS, q_desc, x_k + (gn % NX) * kStep);
+              mma_commit(&ctl.s_full);
+            }
+            if (!wait_bar(&ctl.ds_ready, nph & 1, abort_flag)) { ok = false; break; }
+            ++nph;
+            tc_fence_after_sync();
+            if (j == 0 && pc > 0) {
+              if (!wait_bar(&ctl.acc_empty, (pc - 1) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+            }
+            issue_tmem_a<D>(tmem + kColDQ, tmem + kColDP, x_mn + (gj % NX) * kStep, j > 0);
+            if (gj + NX < total_steps) mma_commit(&ctl.x_empty[gj % NX]);
+            if (more) {
+              if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_qk<D>(tmem + kColDP, o_desc, y_k + (gn % NY) * kStep);
+              mma_commit(&ctl.dp_full);
+              if (gn + NY < total_steps) mma_commit(&ctl.y_empty[gn % NY]);
+            }
+          }
+          if (!ok) break;
+          // the last S_j was loaded too: consume its s_free phase
+          if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
+          ++nsf;
+          if (pc + 1 < total_passes) mma_commit(&ctl.fix_empty);
+          mma_commit(&ctl.acc_ready);
+          g += n;
+          ++pc;
+        }
+      }
+      if (!ok) {
+        mma_commit(&ctl.drain);
+        wait_slow(&ctl.drain, 0, nullptr, kDrainLimitNs);
+      }
+    }
+  } else {
+    // ------------------------------------------- softmax and epilogue ---
+    const int g4 = warp & 3, h = warp >> 2;
+    const int row = g4 * 32 + lane;  // query row of the pass
+    const uint32_t lane_off = static_cast<uint32_t>(g4 * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t ns = 0, nd = 0;
+    int pc = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+      const ItemInfo it = load_item(p.segs, p.work, idx);
+      const int passes = it.b_valid ? 2 : 1;
+      const int seg_end = it.seg_start + it.seg_len;
+      for (int t = 0; t < passes && ok; ++t, ++pc) {
+        const int r0 = it.q0 + t * kSubM;
+        const int q = r0 + row;
+        const bool row_in = q < seg_end;
+        const size_t si = static_cast<size_t>(it.head) * p.total_tokens + q;
+        const float lse2 = row_in ? __ldg(p.lse + si) * kLog2e : 0.0f;
+        const float drow = row_in ? __ldg(p.delta + si) : 0.0f;
+        for (int j = 0; j < it.n_kv; ++j) {
+          if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
+          ++ns;
+          tc_fence_after_sync();
+          uint32_t sr[64];
+          tmem_ld64_sync(tmem + lane_off + kColS + 64 * h, sr);
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.s_free);
+          float pv[64];
+          const int valid = it.seg_len - j * kBlockN - 64 * h;  // keys of this half in the sample
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            pv[c] = ex2_approx(c < valid ? fmaf(__uint_as_float(sr[c]), sl2, -lse2) : -INFINITY);
+          if (!warp_wait_bar(&ctl.dp_full, nd & 1, abort_flag)) { ok = false; break; }
+          ++nd;
+          tc_fence_after_sync();
+          {
+            uint32_t dr[64];
+            tmem_ld64_sync(tmem + lane_off + kColDP + 64 * h, dr);
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              pk[c] = pack_bf16x2(pv[2 * c] * (__uint_as_float(dr[2 * c]) - drow),
+                                  pv[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - drow));
+            tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
+          }
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.ds_ready);
+        }
+        if (!ok) break;
+        if (!warp_wait_bar(&ctl.acc_ready, pc & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after_sync();
+        const size_t orow = (static_cast<size_t>(q) * p.heads + it.head) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          const int col = h * (D / 2) + 32 * c;
+          uint32_t r[32];
+          tmem_ld32_sync(tmem + lane_off + kColDQ + col, r);
+          if (row_in) {
+            float4* dst = reinterpret_cast<float4*>(p.dhat + orow + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(r[4 * v + 0]) * p.scale,
+                                   __uint_as_float(r[4 * v + 1]) * p.scale,
+                                   __uint_as_float(r[4 * v + 2]) * p.scale,
+                                   __uint_as_float(r[4 * v + 3]) * p.scale);
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.acc_empty);
+      }
+    }
+  }
+  bwd_teardown(tmem, warp);
+}
+
+}  // namespace mf

@@ -10,10 +10,13 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/mf_attn.h"
+#include "attention_bwd.cuh"
 #include "packed_attention.cuh"
 #include "qk_prologue.cuh"
+#include "qk_prologue_bwd.cuh"
 
 namespace {
 
@@ -108,6 +111,46 @@ bool prepare_attention_kernel() {
                                    mf::AttnConfig<D>::kSmemBytes) == cudaSuccess;
   });
   return ok[dev];
+}
+
+// Dynamic shared memory of the two backward attention kernels, set once per device.
+template <int D>
+bool prepare_bwd_kernels() {
+  static std::once_flag once[kMaxDevices];
+  static bool ok[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::call_once(once[dev], [dev] {
+    ok[dev] = cudaFuncSetAttribute(mf::attn_bwd_dkdv_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   mf::BwdConfig<D, false>::kSmemBytes) == cudaSuccess &&
+              cudaFuncSetAttribute(mf::attn_bwd_dq_kernel<D>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   mf::BwdConfig<D, true>::kSmemBytes) == cudaSuccess;
+  });
+  return ok[dev];
+}
+
+// Backward workspace: the forward's (q_hat, k_hat, control block), then
+// D [H, T] fp32, dq_hat and dk_hat [T, H, d] fp32 and the per-block partial
+// gamma gradients [blocks, 4, d] fp32.
+struct BwdLayout {
+  WorkspaceLayout fwd;
+  size_t delta, dq_hat, dk_hat, partial, total;
+  int pro_blocks;
+};
+
+bool bwd_layout(int32_t total_tokens, int32_t heads, int32_t head_dim, BwdLayout* b) {
+  if (!layout(total_tokens, heads, head_dim, &b->fwd)) return false;
+  const size_t rows = static_cast<size_t>(total_tokens) * heads;
+  const int tok_per_block = mf::kPrologueThreads / (head_dim / 8);
+  b->pro_blocks = (total_tokens + tok_per_block - 1) / tok_per_block;
+  b->delta = round_up(b->fwd.total, kAlign);
+  b->dq_hat = b->delta + round_up(rows * 4, kAlign);
+  b->dk_hat = b->dq_hat + round_up(rows * head_dim * 4, kAlign);
+  b->partial = b->dk_hat + round_up(rows * head_dim * 4, kAlign);
+  b->total = b->partial + round_up(static_cast<size_t>(b->pro_blocks) * 4 * head_dim * 4, kAlign);
+  return true;
 }
 
 }  // namespace
@@ -339,4 +382,141 @@ extern "C" mf_status mf_get_device_error(void* stream) {
       return MF_ERR_CUDA;
   }
   return static_cast<mf_status>(v);
+}
+
+extern "C" size_t mf_bwd_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim) {
+  BwdLayout b;
+  return bwd_layout(total_tokens, heads, head_dim, &b) ? b.total : 0;
+}
+
+extern "C" mf_status mf_joint_attn_fwd_lse(const void* q, const void* k, const void* v,
+                                           const float* g_q_text, const float* g_q_img,
+                                           const float* g_k_text, const float* g_k_img,
+                                           const int32_t* cu_seqlens_dev,
+                                           const mf_segment* segs_dev, int32_t n_samples,
+                                           const mf_work_item* work_dev, int32_t n_work,
+                                           int32_t total_tokens, int32_t heads, int32_t head_dim,
+                                           float eps, int32_t frame_dims, float softmax_scale,
+                                           void* out, float* lse, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
+  if (!v || !work_dev || !out || !lse || n_work < 1 || !std::isfinite(softmax_scale))
+    return MF_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(out)) return MF_ERR_ALIGNMENT;
+  const size_t bytes = static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * heads * head_dim * 2;
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes)) return MF_ERR_INVALID_ARG;
+  const size_t lse_bytes = static_cast<size_t>(total_tokens > 0 ? total_tokens : 0) * heads * 4;
+  if (overlaps(lse, lse_bytes, q, bytes) || overlaps(lse, lse_bytes, k, bytes))
+    return MF_ERR_INVALID_ARG;
+  mf_status st = mf_qk_prologue_3d(q, k, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev,
+                                   segs_dev, n_samples, total_tokens, heads, head_dim, eps,
+                                   frame_dims, workspace, workspace_bytes, stream);
+  if (st != MF_OK) return st;
+  return packed_attention_impl(v, segs_dev, n_samples, work_dev, n_work, total_tokens, heads,
+                               head_dim, softmax_scale, out, lse, workspace, workspace_bytes,
+                               stream);
+}
+
+extern "C" mf_status mf_joint_attn_bwd(
+    const void* q, const void* k, const void* v, const float* g_q_text, const float* g_q_img,
+    const float* g_k_text, const float* g_k_img, const void* out, const void* dout,
+    const float* lse, const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+    int32_t n_samples, const mf_work_item* work_dev, int32_t n_work, int32_t total_tokens,
+    int32_t heads, int32_t head_dim, float eps, int32_t frame_dims, float softmax_scale, void* dq,
+    void* dk, void* dv, float* dgamma, void* workspace, size_t workspace_bytes, void* stream) {
+  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
+  BwdLayout bl;
+  if (!bwd_layout(total_tokens, heads, head_dim, &bl) || n_samples < 1 || n_work < 1)
+    return MF_ERR_INVALID_ARG;
+  if (!q || !k || !v || !g_q_text || !g_q_img || !g_k_text || !g_k_img || !out || !dout || !lse ||
+      !cu_seqlens_dev || !segs_dev || !work_dev || !dq || !dk || !dv || !dgamma || !workspace)
+    return MF_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps) || !std::isfinite(softmax_scale))
+    return MF_ERR_INVALID_ARG;
+  if (frame_dims < 0 || frame_dims % 4 != 0 || frame_dims > head_dim - 4) return MF_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || (reinterpret_cast<uintptr_t>(dgamma) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MF_ERR_ALIGNMENT;
+  if (workspace_bytes < bl.total) return MF_ERR_WORKSPACE;
+  const size_t bytes = static_cast<size_t>(total_tokens) * heads * head_dim * 2;
+  const size_t lse_bytes = static_cast<size_t>(total_tokens) * heads * 4;
+  const size_t g_bytes = static_cast<size_t>(4) * head_dim * 4;
+  // Outputs must not overlap any input, the workspace or one another.
+  struct Span { const void* p; size_t n; };
+  const Span outs[4] = {{dq, bytes}, {dk, bytes}, {dv, bytes}, {dgamma, g_bytes}};
+  const Span ins[7] = {{q, bytes}, {k, bytes}, {v, bytes}, {out, bytes}, {dout, bytes},
+                       {lse, lse_bytes}, {workspace, bl.total}};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 7; ++j)
+      if (overlaps(outs[i].p, outs[i].n, ins[j].p, ins[j].n)) return MF_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return MF_ERR_INVALID_ARG;
+  }
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // 1. q_hat, k_hat again (the forward's workspace need not have survived).
+  mf_status st = mf_qk_prologue_3d(q, k, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev,
+                                   segs_dev, n_samples, total_tokens, heads, head_dim, eps,
+                                   frame_dims, workspace, workspace_bytes, stream);
+  if (st != MF_OK) return st;
+  const unsigned pro_grid = static_cast<unsigned>(bl.pro_blocks);
+  float* delta = reinterpret_cast<float*>(ws + bl.delta);
+  float* dq_hat = reinterpret_cast<float*>(ws + bl.dq_hat);
+  float* dk_hat = reinterpret_cast<float*>(ws + bl.dk_hat);
+  float* partial = reinterpret_cast<float*>(ws + bl.partial);
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_thd(&tq, ws + bl.fwd.q_hat, total_tokens, heads, head_dim) ||
+      !encode_thd(&tk, ws + bl.fwd.k_hat, total_tokens, heads, head_dim) ||
+      !encode_thd(&tv, v, total_tokens, heads, head_dim) ||
+      !encode_thd(&tdo, dout, total_tokens, heads, head_dim))
+    return MF_ERR_CUDA;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  mf::BwdParams prm;
+  prm.segs = segs_dev;
+  prm.work = work_dev;
+  prm.lse = lse;
+  prm.delta = delta;
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.n_work = n_work;
+  prm.heads = heads;
+  prm.total_tokens = total_tokens;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const int sms = sm_count();
+  if (sms <= 0) return MF_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(n_work < sms ? n_work : sms);
+
+  auto run = [&](auto dtag) -> mf_status {
+    constexpr int D = decltype(dtag)::value;
+    if (!prepare_bwd_kernels<D>()) return MF_ERR_CUDA;
+    // 2. D = rowsum(dO * out)
+    mf::bwd_delta_kernel<D><<<pro_grid, mf::kPrologueThreads, 0, s>>>(
+        static_cast<const uint4*>(out), static_cast<const uint4*>(dout), total_tokens, heads, delta);
+    // 3. dv and dk_hat
+    mf::BwdParams p1 = prm;
+    p1.dhat = dk_hat;
+    mf::attn_bwd_dkdv_kernel<D><<<grid, mf::kBwdThreads, mf::BwdConfig<D, false>::kSmemBytes, s>>>(
+        tq, tk, tv, tdo, p1);
+    // 4. dq_hat
+    mf::BwdParams p2 = prm;
+    p2.dhat = dq_hat;
+    mf::attn_bwd_dq_kernel<D><<<grid, mf::kBwdThreads, mf::BwdConfig<D, true>::kSmemBytes, s>>>(
+        tq, tk, tv, tdo, p2);
+    // 5. back through rotation and norm; 6. gamma gradients
+    mf::qk_prologue_bwd_kernel<D><<<pro_grid, mf::kPrologueThreads, 0, s>>>(
+        static_cast<const uint4*>(q), static_cast<const uint4*>(k),
+        reinterpret_cast<const float4*>(dq_hat), reinterpret_cast<const float4*>(dk_hat), g_q_text,
+        g_q_img, g_k_text, g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps,
+        frame_dims, static_cast<uint4*>(dq), static_cast<uint4*>(dk), partial);
+    const int n_out = 4 * D;
+    mf::dgamma_reduce_kernel<<<(n_out + 255) / 256, 256, 0, s>>>(partial, bl.pro_blocks, n_out,
+                                                                 dgamma);
+    return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
+  };
+  if (head_dim == 128) return run(std::integral_constant<int, 128>{});
+  return run(std::integral_constant<int, 64>{});
 }

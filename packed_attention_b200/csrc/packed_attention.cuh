@@ -125,9 +125,10 @@ struct ItemInfo {
   bool b_valid;
 };
 
-__device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int idx) {
-  const mf_work_item wi = p.work[idx];
-  const mf_segment sg = p.segs[wi.seg];
+__device__ __forceinline__ ItemInfo load_item(const mf_segment* segs, const mf_work_item* work,
+                                              int idx) {
+  const mf_work_item wi = work[idx];
+  const mf_segment sg = segs[wi.seg];
   ItemInfo it;
   it.seg_start = sg.start;
   it.seg_len = sg.len;
@@ -136,6 +137,10 @@ __device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int idx) {
   it.n_kv = (sg.len + kBlockN - 1) / kBlockN;
   it.b_valid = it.q0 + kSubM < sg.start + sg.len;
   return it;
+}
+
+__device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int idx) {
+  return load_item(p.segs, p.work, idx);
 }
 
 struct SharedCtl {

@@ -1,0 +1,180 @@
+"""Backward on the GPU against the oracle's gradients (fp64).
+
+Inputs are the same seeded bf16 tensors for both sides; dL/dout is a seeded
+bf16 tensor. The GPU path recomputes q_hat, k_hat, takes P from the forward's
+log-normaliser, rounds P and dS to bf16 for the tensor cores and the
+gradients once to bf16 at the end; the oracle differentiates the fp64
+forward exactly. Tolerance (relative RMS over all elements of a gradient,
+and max-abs over the gradient's RMS): each gradient passes through about
+three bf16 roundings (2^-9 relative each: q_hat / k_hat or P, dS, the output)
+and sums of ~L terms of random sign, so the relative RMS error sits near
+3 * 2^-9 / sqrt(3) ~ 3.4e-3; the bound is 1e-2 (rel-RMS) with max-abs below
+0.1 of the gradient's RMS.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import packed_attention_b200 as pa
+from packed_attention_b200 import synth
+from packed_attention_b200.workloads import (EXTRA_WORKLOADS, WORKLOADS, Workload, make_inputs,
+                                             random_pack)
+from test_gpu_parity import bf16_to_f64, to_dev
+
+pytestmark = pytest.mark.gpu
+
+REL_RMS_BWD = 1e-2
+MAX_ABS_REL_BWD = 0.1
+NAMES = pa.GAMMA_NAMES
+
+
+def dout_bits(w: Workload):
+    z = synth.normals(w.seed + 1000, synth.STREAM_V, w.total_tokens * w.heads * w.head_dim)
+    return synth.f64_to_bf16_bits(z.reshape(w.total_tokens, w.heads, w.head_dim))
+
+
+def rel_errors(got, ref):
+    diff = got - ref
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    return float(np.max(np.abs(diff))) / rms, float(np.sqrt(np.mean(diff ** 2))) / rms
+
+
+def report(name, errs):
+    path = os.environ.get("MF_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"backward": name, **errs}) + "\n")
+
+
+def run_fwd_bwd(w: Workload, inp, dob, dev):
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=dev)
+    t = to_dev(inp, dev)
+    out, lse = pa.joint_attention_fwd_lse(t["q"], t["k"], t["v"], t, plan, eps=w.eps,
+                                          frame_dims=w.rope_frame_dims)
+    dout = torch.from_numpy(dob.view(np.int16)).view(torch.bfloat16).to(dev)
+    g = pa.joint_attention_bwd(t["q"], t["k"], t["v"], t, plan, out, lse, dout, eps=w.eps,
+                               frame_dims=w.rope_frame_dims)
+    assert pa.device_error() == 0
+    return plan, t, out, lse, g
+
+
+def oracle_grads(w: Workload, inp, dob, heads=None):
+    sel = slice(None) if heads is None else list(heads)
+    q, k, v = (synth.bf16_bits_to_f64(inp[n][:, sel]) for n in ("q", "k", "v"))
+    G = synth.bf16_bits_to_f64(dob[:, sel])
+    gam = {n: inp[n].astype(np.float64) for n in NAMES}
+    return oracle.attn_grad(q, k, v, gam, w.samples, dout=G, eps=w.eps,
+                            frame_dims=w.rope_frame_dims)
+
+
+def check_grads(name, g, ref, heads=None, gammas=True):
+    sel = slice(None) if heads is None else list(heads)
+    errs = {}
+    for key in ("dq", "dk", "dv"):
+        got = bf16_to_f64(g[key])[:, sel]
+        errs[key] = rel_errors(got, ref[key])
+    if gammas:
+        for n in NAMES:
+            errs[n] = rel_errors(g[n].double().cpu().numpy(), ref["dgamma"][n])
+    report(name, errs)
+    for key, (mx, rr) in errs.items():
+        assert rr <= REL_RMS_BWD and mx <= MAX_ABS_REL_BWD, (key, mx, rr)
+
+
+SMALL = [
+    WORKLOADS[0],
+    Workload("ragged_d128", ((77, 12, 20, 1), (0, 9, 15, 1), (5, 1, 1, 1), (200, 8, 8, 2)),
+             heads=3, head_dim=128, seed=11),
+    Workload("ragged_d64", ((13, 10, 13, 1), (128, 1, 1, 1), (0, 16, 8, 1)), heads=2,
+             head_dim=64, seed=12),
+    Workload("tile_edges", ((0, 1, 1, 1), (0, 1, 127, 1), (0, 1, 128, 1), (0, 1, 129, 1),
+                            (1, 16, 16, 1), (0, 1, 257, 1)), heads=2, head_dim=128, seed=13),
+    Workload("frames3d_d128", ((30, 9, 11, 2), (3, 7, 5, 3)), heads=2, head_dim=128, seed=14,
+             rope_frame_dims=16),
+    Workload("frames3d_d64", ((0, 12, 12, 2),), heads=2, head_dim=64, seed=15, rope_frame_dims=8),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_backward_small_packs(cuda_device, w):
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    _, _, out, lse, g = run_fwd_bwd(w, inp, dob, cuda_device)
+    ref = oracle_grads(w, inp, dob)
+    # the forward's log-normaliser, [H, T] on the GPU
+    lse_err = float(np.max(np.abs(lse.double().cpu().numpy() - ref["lse"].T)))
+    report(w.name + "_lse", {"lse_max_abs": lse_err})
+    assert lse_err < 1e-2
+    check_grads(w.name, g, ref)
+
+
+@pytest.mark.parametrize("trial", range(4))
+def test_backward_random_packs(cuda_device, trial):
+    rng = np.random.default_rng(1200 + trial)
+    samples = random_pack(rng, int(rng.integers(1, 6)), 300, 24, 2)
+    d = (64, 128)[trial % 2]
+    w = Workload(f"bwd_random_{trial}", samples, heads=int(rng.integers(1, 4)), head_dim=d,
+                 seed=1250 + trial, rope_frame_dims=(0, 0, 16, 8)[trial])
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    _, _, _, _, g = run_fwd_bwd(w, inp, dob, cuda_device)
+    check_grads(w.name, g, oracle_grads(w, inp, dob))
+
+
+def test_backward_uniform_512sq_all_heads(cuda_device):
+    w = WORKLOADS[1]
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    _, _, _, _, g = run_fwd_bwd(w, inp, dob, cuda_device)
+    check_grads(w.name, g, oracle_grads(w, inp, dob))
+
+
+@pytest.mark.parametrize("key", ["edit_1024sq", "edit_1024sq_rope3d"])
+def test_backward_edit_pack_two_heads(cuda_device, key):
+    w = WORKLOADS[3] if key == "edit_1024sq" else EXTRA_WORKLOADS[key]
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    _, _, _, _, g = run_fwd_bwd(w, inp, dob, cuda_device)
+    heads = (0, w.heads - 1)
+    check_grads(w.name, g, oracle_grads(w, inp, dob, heads), heads, gammas=False)
+
+
+def test_backward_deterministic_and_sample_independent(cuda_device):
+    w = SMALL[1]
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    _, _, _, _, g1 = run_fwd_bwd(w, inp, dob, cuda_device)
+    _, _, _, _, g2 = run_fwd_bwd(w, inp, dob, cuda_device)
+    for key in ("dq", "dk", "dv") + NAMES:
+        assert torch.equal(g1[key].view(torch.int16) if g1[key].dtype == torch.bfloat16 else g1[key],
+                           g2[key].view(torch.int16) if g2[key].dtype == torch.bfloat16 else g2[key]), key
+    # each sample alone gives the same dq, dk, dv bit for bit
+    start = 0
+    for i, L in enumerate(w.seg_lens):
+        tok = np.arange(start, start + L)
+        sub = {n: np.ascontiguousarray(inp[n][tok]) for n in ("q", "k", "v")}
+        sub.update({n: inp[n] for n in NAMES})
+        wi = Workload(f"{w.name}_s{i}", (w.samples[i],), w.heads, w.head_dim, w.seed)
+        _, _, _, _, gi = run_fwd_bwd(wi, sub, np.ascontiguousarray(dob[tok]), cuda_device)
+        for key in ("dq", "dk", "dv"):
+            assert torch.equal(g1[key][start:start + L].view(torch.int16),
+                               gi[key].view(torch.int16)), (i, key)
+        start += L
+
+
+def test_autograd_function_matches_the_direct_call(cuda_device):
+    w = SMALL[2]
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    plan, t, out, lse, g = run_fwd_bwd(w, inp, dob, cuda_device)
+    leaves = [t[n].clone().requires_grad_(True) for n in ("q", "k", "v") + NAMES]
+    o = pa.joint_attention_autograd(*leaves, plan, w.eps)
+    assert torch.equal(o.view(torch.int16), out.view(torch.int16))
+    dout = torch.from_numpy(dob.view(np.int16)).view(torch.bfloat16).to(cuda_device)
+    grads = torch.autograd.grad(o, leaves, dout)
+    for x, key in zip(grads, ("dq", "dk", "dv") + NAMES):
+        assert torch.equal(x, g[key]), key

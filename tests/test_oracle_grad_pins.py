@@ -148,3 +148,29 @@ def test_grad_rejects_bad_arguments():
         oracle.attn_grad(q, k, v, gam, [(1, 2, 2, 0)], dout=G)
     with pytest.raises(ValueError):
         oracle.attn_grad(q, k[:, :, :8], v, gam, samples, dout=G)
+
+
+def test_lse_is_the_log_normaliser_of_the_scores():
+    # log sum_u exp(s_tu) over the sample, from the prologue's q_hat, k_hat
+    samples = [(2, 2, 3, 1), (1, 1, 1, 1), (0, 1, 1, 1)]
+    H, d = 2, 16
+    q, k, v, G, gam = rand_problem(12, samples, H, d)
+    qb, kb = synth.f64_to_bf16_bits(q), synth.f64_to_bf16_bits(k)
+    qv, kv, vv = (synth.bf16_bits_to_f64(x) for x in (qb, kb, synth.f64_to_bf16_bits(v)))
+    g32 = {n: gam[n].astype(np.float32).astype(np.float64) for n in NAMES}
+    lse = oracle.attn_grad(qv, kv, vv, g32, samples)["lse"]
+    qh = oracle.qk_prologue(qb, samples, g32["g_q_text"], g32["g_q_img"])
+    kh = oracle.qk_prologue(kb, samples, g32["g_k_text"], g32["g_k_img"])
+    start = 0
+    for (nt, gh, gw, f) in samples:
+        L = nt + f * gh * gw
+        for h in range(H):
+            s = qh[start:start + L, h] @ kh[start:start + L, h].T / np.sqrt(d)
+            mx = s.max(axis=1, keepdims=True)
+            ref = (mx + np.log(np.exp(s - mx).sum(axis=1, keepdims=True)))[:, 0]
+            np.testing.assert_allclose(lse[start:start + L, h], ref, rtol=0, atol=1e-12)
+        start += L
+    # a one-token sample: lse = its own score
+    t = start - 1
+    for h in range(H):
+        assert lse[t, h] == pytest.approx(qh[t, h] @ kh[t, h] / np.sqrt(d), abs=1e-12)
