@@ -175,6 +175,47 @@ def test_frame_dims_checked_before_any_launch(lib):
     assert lib.mf_joint_attn_fwd_3d(P(0x10008), *base[1:], 16, *tail) == -3
 
 
+def _bwd(lib, **over):
+    """mf_joint_attn_bwd with fake (never dereferenced) pointers."""
+    # Spaced so that nothing overlaps: every test below changes one argument
+    # into an invalid one, and the call must return before any CUDA work.
+    a = dict(q=0x10000, k=0x20000, v=0x30000, gqt=0x40000, gqi=0x40100, gkt=0x40200,
+             gki=0x40300, out=0x50000, dout=0x60000, lse=0x70000, cu=0x71000, segs=0x72000,
+             n=2, work=0x73000, n_work=4, T=152, H=2, d=64, eps=1e-6, F=0, scale=0.0,
+             dq=0x80000, dk=0x90000, dv=0xa0000, dg=0xb0000, ws=0x200000, ws_bytes=1 << 22)
+    a.update(over)
+    P = ctypes.c_void_p
+    return lib.mf_joint_attn_bwd(
+        P(a["q"]), P(a["k"]), P(a["v"]), P(a["gqt"]), P(a["gqi"]), P(a["gkt"]), P(a["gki"]),
+        P(a["out"]), P(a["dout"]), P(a["lse"]), P(a["cu"]), P(a["segs"]), a["n"], P(a["work"]),
+        a["n_work"], a["T"], a["H"], a["d"], a["eps"], a["F"], a["scale"], P(a["dq"]),
+        P(a["dk"]), P(a["dv"]), P(a["dg"]), P(a["ws"]), a["ws_bytes"], None)
+
+
+def test_backward_argument_checks(lib):
+    T, H, d = 152, 2, 64
+    need = lib.mf_bwd_workspace_bytes(T, H, d)
+    rows = T * H
+    r256 = lambda x: (x + 255) // 256 * 256
+    fwd = lib.mf_workspace_bytes(T, H, d)
+    blocks = (T + 31) // 32  # 256 threads, 8 per token at d = 64
+    assert need == r256(fwd) + r256(rows * 4) + 2 * r256(rows * d * 4) + r256(blocks * 4 * d * 4)
+    assert lib.mf_bwd_workspace_bytes(T, H, 96) == 0
+    assert _bwd(lib, d=96) == -2
+    assert _bwd(lib, F=6) == -1
+    assert _bwd(lib, eps=-1.0) == -1
+    assert _bwd(lib, dout=0) == -1
+    assert _bwd(lib, q=0x10008) == -3
+    assert _bwd(lib, dout=0x60004) == -3
+    assert _bwd(lib, lse=0x70002) == -3
+    assert _bwd(lib, dq=0x80008) == -3
+    assert _bwd(lib, ws=0x200010) == -3
+    assert _bwd(lib, ws_bytes=need - 1) == -4
+    assert _bwd(lib, dq=0x10000) == -1          # dq aliases q
+    assert _bwd(lib, dv=0x90000) == -1          # dv aliases dk
+    assert _bwd(lib, dg=0x200100) == -1         # dgamma inside the workspace
+
+
 def test_diagnostic_entry_points_reject_bad_arguments(lib):
     assert lib.mf_selftest_timeout(0, None) == -1
     assert lib.mf_selftest_timeout(2_000_000_000, None) == -1
