@@ -55,6 +55,9 @@ def parse_args():
                     help="workload index 0-4 (default 4), or 'all' for one report line per "
                          "workload (timing only, no e2e / CPU baseline)")
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--train", action="store_true",
+                    help="time the training pass (forward with log-normaliser + backward) of "
+                         "the chosen workload on one GPU and print one JSON line")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -266,6 +269,61 @@ def _median_step_ms(runs, steps, warmup):
     return total, pro, att
 
 
+def training_line(w, key, steps, warmup, peaks, peak_src):
+    """Device time of one training pass over the pack: the forward with its
+    log-normaliser (``mf_joint_attn_fwd_lse``) and the backward
+    (``mf_joint_attn_bwd``), medians over ``steps``. Backward FLOPs are counted
+    as 2.5x the forward's: five products of the forward's size (S again, dP,
+    dV, dK, dQ), the convention of FlashAttention's papers."""
+    import torch
+    import packed_attention_b200 as pa
+    from packed_attention_b200.workloads import make_inputs
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    inp = make_inputs(w)
+    t = _device_inputs(inp, dev, pa, torch)
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=dev)
+    ws = plan.new_workspace()
+    out = torch.empty_like(t["q"])
+    lse = torch.empty(w.heads, w.total_tokens, dtype=torch.float32, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(w.seed)
+    dout = torch.randn(out.shape, generator=gen, device=dev).to(torch.bfloat16)
+    bws = torch.empty(pa.bwd_workspace_bytes(plan), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    fd = w.rope_frame_dims
+
+    def fwd():
+        pa.joint_attention_fwd_lse(t["q"], t["k"], t["v"], t, plan, eps=w.eps, frame_dims=fd,
+                                   out=out, lse=lse, workspace=ws)
+
+    def bwd():
+        pa.joint_attention_bwd(t["q"], t["k"], t["v"], t, plan, out, lse, dout, eps=w.eps,
+                               frame_dims=fd, workspace=bws)
+
+    for _ in range(max(3, warmup)):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in evs:
+        e[0].record(stream)
+        fwd()
+        e[1].record(stream)
+        bwd()
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    if pa.device_error() != 0:
+        raise RuntimeError("kernel reported a device-side error")
+    f_ms = sorted(e[0].elapsed_time(e[1]) for e in evs)[steps // 2]
+    b_ms = sorted(e[1].elapsed_time(e[2]) for e in evs)[steps // 2]
+    return {"workload": w.name, "config": key, "phase": "training",
+            "gflop_forward": w.flops / 1e9, "median_ms_forward_lse": f_ms,
+            "median_ms_backward": b_ms, "tflops_forward": w.flops / (f_ms / 1e3) / 1e12,
+            "tflops_backward": 2.5 * w.flops / (b_ms / 1e3) / 1e12,
+            "frac_sustained_peak_backward": 2.5 * w.flops / (b_ms / 1e3) / 1e12 / sustained,
+            "tokens_per_s_training": w.total_tokens / ((f_ms + b_ms) / 1e3), "peaks": peak_src}
+
+
 def report_all(args):
     """One JSON line per workload: device time of both stages, TFLOP/s, tokens/s,
     fraction of the measured peaks (single GPU). Then one line per packed-CFG
@@ -295,50 +353,11 @@ def report_all(args):
             "prologue_gbs": 8 * T * H * d / (pro / 1e3) / 1e9,
             "rope_frame_dims": w.rope_frame_dims, "peaks": peak_src}), flush=True)
 
-    # Training: forward with the log-normaliser, then the backward (one call
-    # each). Backward FLOPs counted as 2.5x the forward's (five products of
-    # the forward's size: S recomputed, dP, dV, dK, dQ).
+    # Training: forward with the log-normaliser, then the backward.
     for key, w in [(1, WORKLOADS[1]), (2, WORKLOADS[2]), (3, WORKLOADS[3]), (4, WORKLOADS[4]),
                    ("edit_1024sq_rope3d", EXTRA_WORKLOADS["edit_1024sq_rope3d"])]:
-        inp = make_inputs(w)
-        t, plan, ws, out, eps, fd = prepare(w, inp)
-        lse = torch.empty(w.heads, w.total_tokens, dtype=torch.float32, device=dev)
-        dout = torch.randn_like(out)
-        bws = torch.empty(pa.bwd_workspace_bytes(plan), dtype=torch.uint8, device=dev)
-        stream = torch.cuda.current_stream()
-
-        def fwd():
-            pa.joint_attention_fwd_lse(t["q"], t["k"], t["v"], t, plan, eps=eps, frame_dims=fd,
-                                       out=out, lse=lse, workspace=ws)
-
-        def bwd():
-            pa.joint_attention_bwd(t["q"], t["k"], t["v"], t, plan, out, lse, dout, eps=eps,
-                                   frame_dims=fd, workspace=bws)
-
-        for _ in range(max(3, args.warmup)):
-            fwd()
-            bwd()
-        torch.cuda.synchronize()
-        K = max(5, args.steps // 5)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-        for e in evs:
-            e[0].record(stream)
-            fwd()
-            e[1].record(stream)
-            bwd()
-            e[2].record(stream)
-        torch.cuda.synchronize()
-        if pa.device_error() != 0:
-            raise RuntimeError("kernel reported a device-side error")
-        f_ms = sorted(e[0].elapsed_time(e[1]) for e in evs)[K // 2]
-        b_ms = sorted(e[1].elapsed_time(e[2]) for e in evs)[K // 2]
-        print(json.dumps({
-            "workload": w.name, "config": key, "phase": "training", "gflop_forward": w.flops / 1e9,
-            "median_ms_forward_lse": f_ms, "median_ms_backward": b_ms,
-            "tflops_forward": w.flops / (f_ms / 1e3) / 1e12,
-            "tflops_backward": 2.5 * w.flops / (b_ms / 1e3) / 1e12,
-            "frac_sustained_peak_backward": 2.5 * w.flops / (b_ms / 1e3) / 1e12 / sustained,
-            "peaks": peak_src}), flush=True)
+        print(json.dumps(training_line(w, key, max(5, args.steps // 5), args.warmup, peaks,
+                                       peak_src)), flush=True)
 
     for name, cp in CFG_PACKS.items():
         w = cp.packed()
@@ -370,6 +389,13 @@ def main():
         report_all(args)
         return
     w = WORKLOADS[int(args.config)]
+    if args.train:
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        peaks, peak_src = load_peaks()
+        print(json.dumps(training_line(w, int(args.config), args.steps, args.warmup, peaks,
+                                       peak_src)), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args, w)
         return
