@@ -26,27 +26,32 @@
 //
 // dK/dV kernel, per pass: 128 key rows; K_hat and V stay in shared memory and
 // every query step j brings Q_hat_j and dO_j (two rings). TMEM columns:
-//   S^T = K_hat Q_hat_j^T [0,128)   P^T (bf16) over its columns [0,32) and [64,96)
+//   S^T = K_hat Q_hat_j^T [0,128)
 //   dP^T = V dO_j^T     [128,256)   dS^T (bf16) over [128,160) and [192,224)
 //   dV accumulator      [256,256+d)
 //   dK accumulator      [384,384+d)
-// MMA order per step: dV_j, S^T_{j+1}, dK_j, dP^T_{j+1}. The softmax computes
-// P^T_{j+1} while the tensor core runs dK_j and dP^T_{j+1}, and dS^T_{j+1}
-// while it runs dV_{j+1} and S^T_{j+2}. MMAs of one thread execute in issue
-// order, so S^T_{j+1} overwrites P^T_j only after dV_j has read it (and
-// dP^T_{j+1} overwrites dS^T_j only after dK_j).
+// P^T (bf16) goes to shared memory (128-byte swizzled, K-major), the A
+// operand of dV += P^T dO_j. S^T_{j+1} is issued as soon as every softmax
+// warp holds S^T_j in registers, so no MMA waits on the exponentials of its
+// own step: per step the tensor core runs S^T_{j+1}, dV_j, dK_j, dP^T_{j+1}
+// while the softmax computes P^T_{j+1} and then dS^T_{j+1}. MMAs of one
+// thread execute in issue order, so dP^T_{j+1} overwrites dS^T_j only after
+// dK_j has read it.
 //
 // dQ kernel, per pass: 128 query rows; Q_hat and dO stay, every key step
-// brings K_hat_j and V_j. TMEM: S [0,128), dP [128,256) with dS (bf16) written
-// over its columns [128,160) and [192,224), dQ accumulator [256,256+d). S_{j+1}
-// is issued as soon as every softmax warp has loaded S_j into registers;
-// order per step: S_{j+1}, dQ_j, dP_{j+1}.
+// brings K_hat_j and V_j. TMEM: S [0,128), dP in two buffers [128,256) and
+// [384,512) with dS (bf16) written over the first 32 columns of each 64-column
+// half, dQ accumulator [256,256+d). Per step: S_{j+1} and dP_{j+1} as soon as
+// the softmax holds S_j, then dQ_j once dS_j is written.
 #pragma once
 
 #include "packed_attention.cuh"
 
 namespace mf {
 
+// Warps 0-7 softmax and epilogue, 8 TMA producer, 9 MMA issuer. Ten warps
+// put three on two of the SM's four sub-partitions, which caps a thread at
+// 168 registers.
 constexpr int kBwdThreads = 320;
 constexpr int kBwdProducerWarp = 8;
 constexpr int kBwdMmaWarp = 9;
@@ -58,9 +63,11 @@ template <int D, bool kDq>
 struct BwdConfig {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kSubM * D * 2;
+  static constexpr int kPTileBytes = kSubM * kBlockN * 2;  // P^T of one step (dK/dV kernel)
   static constexpr int kRingX = (kDq || D == 64) ? 3 : 2;
   static constexpr int kRingY = 2;
-  static constexpr int kSmemBytes = kTileBytes * (2 + kRingX + kRingY) + 1024;
+  static constexpr int kSmemBytes =
+      kTileBytes * (2 + kRingX + kRingY) + (kDq ? 0 : kPTileBytes) + 1024;
 };
 
 struct BwdParams {
@@ -81,8 +88,8 @@ struct BwdCtl {
   uint64_t fix_full, fix_empty;
   uint64_t x_full[3], x_empty[3];
   uint64_t y_full[2], y_empty[2];
-  uint64_t s_full, s_free, dp_full;
-  uint64_t p_ready, ds_ready;
+  uint64_t s_full, s_free, dp_full[2];
+  uint64_t p_ready, p_free, ds_ready;
   uint64_t acc_ready, acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
@@ -102,6 +109,25 @@ __device__ __forceinline__ void issue_tmem_a(uint32_t d_tmem, uint32_t a_tmem, u
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// D (+)= A (shared, K-major, 128-byte swizzle: 128 rows x 128 K in two
+// 64-column boxes) * B (shared, MN-major [K = 128 rows][N = D]).
+template <int D>
+__device__ __forceinline__ void issue_smem_a(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             bool accumulate) {
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ss(d_tmem, a_desc + static_cast<uint64_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4),
+           b_desc + static_cast<uint64_t>(kk * (2048 >> 4)), kIdesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Column c (0..63) of a warp's half: value held by lane c / 2, low or high
+// element (the layout in which the softmax warps hold per-column statistics).
+__device__ __forceinline__ uint64_t col_pair(float lo, float hi, int c2) {
+  return f32x2(__shfl_sync(0xffffffffu, lo, c2), __shfl_sync(0xffffffffu, hi, c2));
+}
+
 template <int D, bool kDq>
 __device__ __forceinline__ void bwd_init(BwdCtl& ctl, int warp) {
   if (threadIdx.x == 0) {
@@ -117,8 +143,10 @@ __device__ __forceinline__ void bwd_init(BwdCtl& ctl, int warp) {
     }
     mbar_init(&ctl.s_full, 1);
     mbar_init(&ctl.s_free, 8);
-    mbar_init(&ctl.dp_full, 1);
+    mbar_init(&ctl.dp_full[0], 1);
+    mbar_init(&ctl.dp_full[1], 1);
     mbar_init(&ctl.p_ready, 8);
+    mbar_init(&ctl.p_free, 1);
     mbar_init(&ctl.ds_ready, 8);
     mbar_init(&ctl.acc_ready, 1);
     mbar_init(&ctl.acc_empty, 8);
@@ -230,13 +258,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ BwdCtl ctl;
-  __shared__ __align__(16) float s_stat[8][2][64];  // per softmax warp: lse (log2) and D
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sK = smem;              // fixed: K_hat then V
-  uint8_t* sV = smem + kTile;
-  uint8_t* sX = smem + 2 * kTile;  // ring of Q_hat
-  uint8_t* sY = sX + NX * kTile;   // ring of dO
+  uint8_t* sP = smem;                  // P^T of the current step (two 64-query boxes)
+  uint8_t* sK = smem + Cfg::kPTileBytes;  // fixed: K_hat then V
+  uint8_t* sV = sK + kTile;
+  uint8_t* sX = sK + 2 * kTile;        // ring of Q_hat
+  uint8_t* sY = sX + NX * kTile;       // ring of dO
   volatile int32_t* abort_flag = &ctl.abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -255,6 +283,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bwd_producer<D, false>(p, ctl, sK, sX, sY, &tmap_k, &tmap_v, &tmap_q, &tmap_do, abort_flag);
   } else if (warp == kBwdMmaWarp) {
     if (lane == 0) {
+      const uint64_t p_desc = smem_desc_sw128(smem_addr(sP), 16, 1024);       // P^T as A of dV
       const uint64_t k_desc = smem_desc_sw128(smem_addr(sK), 16, 1024);
       const uint64_t v_desc = smem_desc_sw128(smem_addr(sV), 16, 1024);
       const uint64_t x_k = smem_desc_sw128(smem_addr(sX), 16, 1024);          // Q_hat as B of S^T
@@ -265,7 +294,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int total_passes, total_steps;
       bwd_counts(p, total_passes, total_steps);
       int pc = 0, g = 0;
-      uint32_t nph = 0;
+      uint32_t nph = 0, nsf = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
         const ItemInfo it = load_item(p.segs, p.work, idx);
@@ -281,10 +310,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!wait_bar(&ctl.y_full[g % NY], (g / NY) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
           issue_qk<D>(tmem + kColDP, v_desc, y_k + (g % NY) * kStep);
-          mma_commit(&ctl.dp_full);
+          mma_commit(&ctl.dp_full[0]);
           for (int j = 0; j < n && ok; ++j) {
             const int gj = g + j, gn = gj + 1;
             const bool more = j + 1 < n;
+            if (more) {
+              // S^T_{j+1} as soon as every softmax warp holds S^T_j
+              if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
+              ++nsf;
+              if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_qk<D>(tmem + kColS, k_desc, x_k + (gn % NX) * kStep);
+              mma_commit(&ctl.s_full);
+            }
             if (!wait_bar(&ctl.p_ready, nph & 1, abort_flag)) { ok = false; break; }
             tc_fence_after_sync();
             if (j == 0 && pc > 0) {
@@ -292,14 +330,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (!wait_bar(&ctl.acc_empty, (pc - 1) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
             }
-            issue_tmem_a<D>(tmem + kColDV, tmem + kColS, y_mn + (gj % NY) * kStep, j > 0);
+            issue_smem_a<D>(tmem + kColDV, p_desc, y_mn + (gj % NY) * kStep, j > 0);
+            mma_commit(&ctl.p_free);
             if (gj + NY < total_steps) mma_commit(&ctl.y_empty[gj % NY]);
-            if (more) {
-              if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after_sync();
-              issue_qk<D>(tmem + kColS, k_desc, x_k + (gn % NX) * kStep);
-              mma_commit(&ctl.s_full);
-            }
             if (!wait_bar(&ctl.ds_ready, nph & 1, abort_flag)) { ok = false; break; }
             ++nph;
             tc_fence_after_sync();
@@ -309,10 +342,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
               issue_qk<D>(tmem + kColDP, v_desc, y_k + (gn % NY) * kStep);
-              mma_commit(&ctl.dp_full);
+              mma_commit(&ctl.dp_full[0]);
             }
           }
           if (!ok) break;
+          // the last S^T of the pass was loaded too: consume its s_free phase
+          if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
+          ++nsf;
           if (pc + 1 < total_passes) mma_commit(&ctl.fix_empty);
           mma_commit(&ctl.acc_ready);
           g += n;
@@ -329,10 +365,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int g4 = warp & 3, h = warp >> 2;  // TMEM lane quarter, column half
     const int row = g4 * 32 + lane;          // key row of the pass
     const uint32_t lane_off = static_cast<uint32_t>(g4 * 32) << 16;
-    const float sl2 = p.scale_log2;
-    float* st_l = s_stat[warp][0];
-    float* st_d = s_stat[warp][1];
-    uint32_t ns = 0, nd = 0;
+    const uint64_t sl2x2 = f32x2(p.scale_log2, p.scale_log2);
+    // this thread's row of the P^T tile: box h, 128-byte row `row`, 16-byte
+    // chunks at (c ^ (row % 8)) under the 128-byte swizzle
+    uint8_t* p_row = sP + h * kBoxBytes + row * 128;
+    const int swz = row & 7;
+    uint32_t ns = 0, nd = 0, gstep = 0;
     int pc = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
@@ -340,70 +378,78 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int passes = it.b_valid ? 2 : 1;
       const int seg_end = it.seg_start + it.seg_len;
       const size_t stat0 = static_cast<size_t>(it.head) * p.total_tokens;
+      // -lse (log2 units) and D of query columns 2*lane, 2*lane+1 of this
+      // warp's half of step j; queries past the sample end get -lse = -inf
+      // (P = 0) and D = 0.
+      auto load_stats = [&](int j, float& nl0, float& nl1, float& d0, float& d1) {
+        const int q0 = it.seg_start + j * kBlockN + 64 * h + 2 * lane;
+        nl0 = q0 < seg_end ? -__ldg(p.lse + stat0 + q0) * kLog2e : -INFINITY;
+        nl1 = q0 + 1 < seg_end ? -__ldg(p.lse + stat0 + q0 + 1) * kLog2e : -INFINITY;
+        d0 = q0 < seg_end ? __ldg(p.delta + stat0 + q0) : 0.0f;
+        d1 = q0 + 1 < seg_end ? __ldg(p.delta + stat0 + q0 + 1) : 0.0f;
+      };
       for (int t = 0; t < passes && ok; ++t, ++pc) {
         const int r0 = it.q0 + t * kSubM;
         const bool row_in = r0 + row < seg_end;
-        for (int j = 0; j < it.n_kv; ++j) {
-          // lse (log2 units) and D of this warp's 64 queries; queries past
-          // the sample end get lse = +inf, hence P = 0 and dS = 0.
-          {
-            const int qa = it.seg_start + j * kBlockN + 64 * h + lane, qb = qa + 32;
-            const float la = qa < seg_end ? __ldg(p.lse + stat0 + qa) * kLog2e : INFINITY;
-            const float lb = qb < seg_end ? __ldg(p.lse + stat0 + qb) * kLog2e : INFINITY;
-            const float da = qa < seg_end ? __ldg(p.delta + stat0 + qa) : 0.0f;
-            const float db = qb < seg_end ? __ldg(p.delta + stat0 + qb) : 0.0f;
-            __syncwarp();
-            st_l[lane] = la;
-            st_l[lane + 32] = lb;
-            st_d[lane] = da;
-            st_d[lane + 32] = db;
-            __syncwarp();
-          }
+        float nl0, nl1, d0, d1;
+        load_stats(0, nl0, nl1, d0, d1);
+        for (int j = 0; j < it.n_kv; ++j, ++gstep) {
           if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
           ++ns;
           tc_fence_after_sync();
-          float pv[64];
-          {
-            uint32_t sr[64];
-            tmem_ld64_sync(tmem + lane_off + kColS + 64 * h, sr);
-            uint32_t pk[32];
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-              const float4 l = reinterpret_cast<const float4*>(st_l)[c4];
-              pv[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), sl2, -l.x));
-              pv[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l.y));
-              pv[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l.z));
-              pv[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l.w));
-              pk[2 * c4] = pack_bf16x2(pv[4 * c4 + 0], pv[4 * c4 + 1]);
-              pk[2 * c4 + 1] = pack_bf16x2(pv[4 * c4 + 2], pv[4 * c4 + 3]);
-            }
-            tmem_st32_sync(tmem + lane_off + kColS + 64 * h, pk);
-          }
+          uint32_t sr[64];
+          tmem_ld64_sync(tmem + lane_off + kColS + 64 * h, sr);
           tc_fence_before_sync();
           __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.s_free);
+          // next step's statistics, in flight while this step computes
+          float nnl0 = 0.f, nnl1 = 0.f, nd0 = 0.f, nd1 = 0.f;
+          if (j + 1 < it.n_kv) load_stats(j + 1, nnl0, nnl1, nd0, nd1);
+          uint64_t pp[32];
+          uint32_t pk[32];
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])),
+                                         sl2x2, col_pair(nl0, nl1, c2));
+            float x0, x1;
+            f32x2_split(x, x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            pp[c2] = f32x2(p0, p1);
+            pk[c2] = pack_bf16x2(p0, p1);
+          }
+          // P^T_j into shared memory once dV_{j-1} has read P^T_{j-1}
+          if (!warp_wait_bar(&ctl.p_free, (gstep & 1) ^ 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(p_row + ((c ^ swz) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
           if (lane == 0) mbar_arrive(&ctl.p_ready);
-          if (!warp_wait_bar(&ctl.dp_full, nd & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait_bar(&ctl.dp_full[0], nd & 1, abort_flag)) { ok = false; break; }
           ++nd;
           tc_fence_after_sync();
-          {
-            uint32_t dr[64];
-            tmem_ld64_sync(tmem + lane_off + kColDP + 64 * h, dr);
-            uint32_t pk[32];
+          // dS in two halves of 32 columns (keeps dP and P in registers together)
 #pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-              const float4 dd = reinterpret_cast<const float4*>(st_d)[c4];
-              const float d0 = pv[4 * c4 + 0] * (__uint_as_float(dr[4 * c4 + 0]) - dd.x);
-              const float d1 = pv[4 * c4 + 1] * (__uint_as_float(dr[4 * c4 + 1]) - dd.y);
-              const float d2 = pv[4 * c4 + 2] * (__uint_as_float(dr[4 * c4 + 2]) - dd.z);
-              const float d3 = pv[4 * c4 + 3] * (__uint_as_float(dr[4 * c4 + 3]) - dd.w);
-              pk[2 * c4] = pack_bf16x2(d0, d1);
-              pk[2 * c4 + 1] = pack_bf16x2(d2, d3);
+          for (int half = 0; half < 2; ++half) {
+            uint32_t dr[32];
+            tmem_ld32_sync(tmem + lane_off + kColDP + 64 * h + 32 * half, dr);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c2 = 16 * half + i;
+              const uint64_t ds = mul_f32x2(
+                  pp[c2], sub_f32x2(f32x2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
+                                    col_pair(d0, d1, c2)));
+              float a, b;
+              f32x2_split(ds, a, b);
+              pk[c2] = pack_bf16x2(a, b);
             }
-            tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
           }
+          tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl.ds_ready);
+          nl0 = nnl0; nl1 = nnl1; d0 = nd0; d1 = nd1;
         }
         if (!ok) break;
         // ---- epilogue: dv (bf16) and dk_hat = scale * acc (fp32) rows ----
@@ -457,7 +503,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
   using Cfg = BwdConfig<D, true>;
   constexpr int NX = Cfg::kRingX, NY = Cfg::kRingY, kTile = Cfg::kTileBytes;
-  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+  constexpr uint32_t kColS = 0, kColDQ = 256;
+  constexpr uint32_t kColDP[2] = {128, 384};
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ BwdCtl ctl;
@@ -509,20 +556,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_commit(&ctl.s_full);
           if (!wait_bar(&ctl.y_full[g % NY], (g / NY) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_qk<D>(tmem + kColDP, o_desc, y_k + (g % NY) * kStep);
-          mma_commit(&ctl.dp_full);
+          issue_qk<D>(tmem + kColDP[0], o_desc, y_k + (g % NY) * kStep);
+          mma_commit(&ctl.dp_full[0]);
           if (g + NY < total_steps) mma_commit(&ctl.y_empty[g % NY]);
           for (int j = 0; j < n && ok; ++j) {
             const int gj = g + j, gn = gj + 1;
             const bool more = j + 1 < n;
             if (more) {
-              // S_{j+1} as soon as every softmax warp holds S_j in registers
+              // S_{j+1} and dP_{j+1} as soon as every softmax warp holds S_j
+              // (dP_{j+1} goes to the other buffer; the one it overwrites was
+              // read by dQ_{j-1}, issued before)
               if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
               ++nsf;
               if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
               issue_qk<D>(tmem + kColS, q_desc, x_k + (gn % NX) * kStep);
               mma_commit(&ctl.s_full);
+              if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_qk<D>(tmem + kColDP[(j + 1) & 1], o_desc, y_k + (gn % NY) * kStep);
+              mma_commit(&ctl.dp_full[(j + 1) & 1]);
+              if (gn + NY < total_steps) mma_commit(&ctl.y_empty[gn % NY]);
             }
             if (!wait_bar(&ctl.ds_ready, nph & 1, abort_flag)) { ok = false; break; }
             ++nph;
@@ -531,15 +585,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (!wait_bar(&ctl.acc_empty, (pc - 1) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
             }
-            issue_tmem_a<D>(tmem + kColDQ, tmem + kColDP, x_mn + (gj % NX) * kStep, j > 0);
+            issue_tmem_a<D>(tmem + kColDQ, tmem + kColDP[j & 1], x_mn + (gj % NX) * kStep, j > 0);
             if (gj + NX < total_steps) mma_commit(&ctl.x_empty[gj % NX]);
-            if (more) {
-              if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after_sync();
-              issue_qk<D>(tmem + kColDP, o_desc, y_k + (gn % NY) * kStep);
-              mma_commit(&ctl.dp_full);
-              if (gn + NY < total_steps) mma_commit(&ctl.y_empty[gn % NY]);
-            }
           }
           if (!ok) break;
           // the last S_j was loaded too: consume its s_free phase
@@ -561,8 +608,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int g4 = warp & 3, h = warp >> 2;
     const int row = g4 * 32 + lane;  // query row of the pass
     const uint32_t lane_off = static_cast<uint32_t>(g4 * 32) << 16;
-    const float sl2 = p.scale_log2;
-    uint32_t ns = 0, nd = 0;
+    const uint64_t sl2x2 = f32x2(p.scale_log2, p.scale_log2);
+    uint32_t ns = 0, nd[2] = {0, 0};
     int pc = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
@@ -574,8 +621,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int q = r0 + row;
         const bool row_in = q < seg_end;
         const size_t si = static_cast<size_t>(it.head) * p.total_tokens + q;
-        const float lse2 = row_in ? __ldg(p.lse + si) * kLog2e : 0.0f;
+        const float nl = row_in ? -__ldg(p.lse + si) * kLog2e : 0.0f;
         const float drow = row_in ? __ldg(p.delta + si) : 0.0f;
+        const uint64_t nl2 = f32x2(nl, nl), d2 = f32x2(drow, drow);
         for (int j = 0; j < it.n_kv; ++j) {
           if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
           ++ns;
@@ -585,23 +633,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl.s_free);
-          float pv[64];
           const int valid = it.seg_len - j * kBlockN - 64 * h;  // keys of this half in the sample
+          if (valid < 64) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            pv[c] = ex2_approx(c < valid ? fmaf(__uint_as_float(sr[c]), sl2, -lse2) : -INFINITY);
-          if (!warp_wait_bar(&ctl.dp_full, nd & 1, abort_flag)) { ok = false; break; }
-          ++nd;
+            for (int c = 0; c < 64; ++c)
+              if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+          }
+          uint64_t pp[32];
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])),
+                                         sl2x2, nl2);
+            float x0, x1;
+            f32x2_split(x, x0, x1);
+            pp[c2] = f32x2(ex2_approx(x0), ex2_approx(x1));
+          }
+          const int b = j & 1;
+          if (!warp_wait_bar(&ctl.dp_full[b], nd[b] & 1, abort_flag)) { ok = false; break; }
+          ++nd[b];
           tc_fence_after_sync();
           {
-            uint32_t dr[64];
-            tmem_ld64_sync(tmem + lane_off + kColDP + 64 * h, dr);
             uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              pk[c] = pack_bf16x2(pv[2 * c] * (__uint_as_float(dr[2 * c]) - drow),
-                                  pv[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - drow));
-            tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
+            for (int half = 0; half < 2; ++half) {
+              uint32_t dr[32];
+              tmem_ld32_sync(tmem + lane_off + kColDP[b] + 64 * h + 32 * half, dr);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int c2 = 16 * half + i;
+                const uint64_t ds = mul_f32x2(
+                    pp[c2], sub_f32x2(f32x2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])), d2));
+                float a, bb;
+                f32x2_split(ds, a, bb);
+                pk[c2] = pack_bf16x2(a, bb);
+              }
+            }
+            tmem_st32_sync(tmem + lane_off + kColDP[b] + 64 * h, pk);
           }
           tc_fence_before_sync();
           __syncwarp();
