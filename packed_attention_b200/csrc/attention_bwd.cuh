@@ -24,25 +24,32 @@
 // mbarrier waits throughout. A work item of the forward's list (256 rows of
 // one head of one sample) is done as two passes of 128 rows.
 //
+// Shared-memory bandwidth, not the tensor pipe, is what these kernels must
+// budget: an MMA of 128 x 128 x 16 with both operands in shared memory reads
+// 8 KB in its 64 cycles, the whole 128 B/clk the SM has, while one with A in
+// TMEM reads 4 KB. Operands reused across a pass therefore sit in TMEM where
+// there is room, and so do P and dS.
+//
 // dK/dV kernel, per pass: 128 key rows; K_hat and V stay in shared memory and
-// every query step j brings Q_hat_j and dO_j (two rings). TMEM columns:
-//   S^T = K_hat Q_hat_j^T [0,128)
+// every query step j brings Q_hat_j (3-stage ring) and dO_j (2-stage ring).
+// TMEM columns:
+//   S^T = K_hat Q_hat_j^T [0,128)   P^T (bf16) over [0,32) and [64,96)
 //   dP^T = V dO_j^T     [128,256)   dS^T (bf16) over [128,160) and [192,224)
 //   dV accumulator      [256,256+d)
 //   dK accumulator      [384,384+d)
-// P^T (bf16) goes to shared memory (128-byte swizzled, K-major), the A
-// operand of dV += P^T dO_j. S^T_{j+1} is issued as soon as every softmax
-// warp holds S^T_j in registers, so no MMA waits on the exponentials of its
-// own step: per step the tensor core runs S^T_{j+1}, dV_j, dK_j, dP^T_{j+1}
-// while the softmax computes P^T_{j+1} and then dS^T_{j+1}. MMAs of one
-// thread execute in issue order, so dP^T_{j+1} overwrites dS^T_j only after
-// dK_j has read it.
+// P^T and dS^T are the TMEM A operands of dV += P^T dO_j and dK += dS^T Q_j.
+// MMA order per step: dV_j, S^T_{j+1}, dK_j, dP^T_{j+1}: the exponentials of
+// step j+1 overlap dK_j and dP^T_{j+1}, its dS overlaps dV_{j+1} and
+// S^T_{j+2}. MMAs of one thread execute in issue order, so S^T_{j+1}
+// overwrites P^T_j only after dV_j has read it (and dP^T_{j+1} dS^T_j only
+// after dK_j).
 //
-// dQ kernel, per pass: 128 query rows; Q_hat and dO stay, every key step
-// brings K_hat_j and V_j. TMEM: S [0,128), dP in two buffers [128,256) and
-// [384,512) with dS (bf16) written over the first 32 columns of each 64-column
-// half, dQ accumulator [256,256+d). Per step: S_{j+1} and dP_{j+1} as soon as
-// the softmax holds S_j, then dQ_j once dS_j is written.
+// dQ kernel, per pass: 128 query rows. Q_hat and dO are read once per pass
+// into TMEM (the A operands of S and dP); every key step brings K_hat_j
+// (4-stage ring) and V_j (3-stage ring). TMEM: S [0,128), dP [128,256) with
+// dS (bf16) over [128,160) and [192,224), dQ accumulator [256,256+d), Q_hat
+// [384,384+d/2), dO [448,448+d/2). Per step: S_{j+1} as soon as every
+// softmax warp holds S_j in registers, dQ_j once dS_j is written, dP_{j+1}.
 #pragma once
 
 #include "packed_attention.cuh"
@@ -57,17 +64,18 @@ constexpr int kBwdProducerWarp = 8;
 constexpr int kBwdMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// kRingX: the operand held longest (Q_hat in dK/dV, K_hat in dQ);
-// kRingY: the one released after its first MMA (dO in dK/dV, V in dQ).
+// kFix: tiles kept in shared memory for a whole pass (K_hat, V in dK/dV; the
+// dQ kernel keeps Q_hat and dO in TMEM instead). kRingX: the ring operand
+// held longest (Q_hat in dK/dV, K_hat in dQ); kRingY: the one released after
+// its first MMA (dO in dK/dV, V in dQ).
 template <int D, bool kDq>
 struct BwdConfig {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kSubM * D * 2;
-  static constexpr int kPTileBytes = kSubM * kBlockN * 2;  // P^T of one step (dK/dV kernel)
-  static constexpr int kRingX = (kDq || D == 64) ? 3 : 2;
-  static constexpr int kRingY = 2;
-  static constexpr int kSmemBytes =
-      kTileBytes * (2 + kRingX + kRingY) + (kDq ? 0 : kPTileBytes) + 1024;
+  static constexpr int kFix = kDq ? 0 : 2;
+  static constexpr int kRingX = kDq ? 4 : 3;
+  static constexpr int kRingY = kDq ? 3 : 2;
+  static constexpr int kSmemBytes = kTileBytes * (kFix + kRingX + kRingY) + 1024;
 };
 
 struct BwdParams {
@@ -77,6 +85,8 @@ struct BwdParams {
   const float* delta;     // [heads, total_tokens]
   float* dhat;            // fp32 [total_tokens, heads, D]: dk_hat or dq_hat
   __nv_bfloat16* dv;      // bf16 [total_tokens, heads, D] (dK/dV kernel)
+  const uint4* q_rows;    // q_hat [total_tokens, heads, D] (dQ kernel: read into TMEM)
+  const uint4* do_rows;   // dO, same layout (dQ kernel)
   int n_work;
   int heads;
   int total_tokens;
@@ -86,10 +96,10 @@ struct BwdParams {
 
 struct BwdCtl {
   uint64_t fix_full, fix_empty;
-  uint64_t x_full[3], x_empty[3];
-  uint64_t y_full[2], y_empty[2];
-  uint64_t s_full, s_free, dp_full[2];
-  uint64_t p_ready, p_free, ds_ready;
+  uint64_t x_full[4], x_empty[4];
+  uint64_t y_full[3], y_empty[3];
+  uint64_t s_full, s_free, dp_full;
+  uint64_t p_ready, ds_ready, q_ready;
   uint64_t acc_ready, acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
@@ -109,19 +119,6 @@ __device__ __forceinline__ void issue_tmem_a(uint32_t d_tmem, uint32_t a_tmem, u
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// D (+)= A (shared, K-major, 128-byte swizzle: 128 rows x 128 K in two
-// 64-column boxes) * B (shared, MN-major [K = 128 rows][N = D]).
-template <int D>
-__device__ __forceinline__ void issue_smem_a(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                             bool accumulate) {
-  constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, D, 0, 1);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_ss(d_tmem, a_desc + static_cast<uint64_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4),
-           b_desc + static_cast<uint64_t>(kk * (2048 >> 4)), kIdesc,
-           (accumulate || kk > 0) ? 1u : 0u);
-}
-
 // Column c (0..63) of a warp's half: value held by lane c / 2, low or high
 // element (the layout in which the softmax warps hold per-column statistics).
 __device__ __forceinline__ uint64_t col_pair(float lo, float hi, int c2) {
@@ -133,21 +130,20 @@ __device__ __forceinline__ void bwd_init(BwdCtl& ctl, int warp) {
   if (threadIdx.x == 0) {
     mbar_init(&ctl.fix_full, 1);
     mbar_init(&ctl.fix_empty, 1);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&ctl.x_full[s], 1);
       mbar_init(&ctl.x_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(&ctl.y_full[s], 1);
       mbar_init(&ctl.y_empty[s], 1);
     }
     mbar_init(&ctl.s_full, 1);
     mbar_init(&ctl.s_free, 8);
-    mbar_init(&ctl.dp_full[0], 1);
-    mbar_init(&ctl.dp_full[1], 1);
+    mbar_init(&ctl.dp_full, 1);
     mbar_init(&ctl.p_ready, 8);
-    mbar_init(&ctl.p_free, 1);
     mbar_init(&ctl.ds_ready, 8);
+    mbar_init(&ctl.q_ready, 8);
     mbar_init(&ctl.acc_ready, 1);
     mbar_init(&ctl.acc_empty, 8);
     mbar_init(&ctl.drain, 1);
@@ -192,14 +188,16 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BwdCtl& ctl, ui
     const int passes = it.b_valid ? 2 : 1;
     for (int t = 0; t < passes && ok; ++t) {
       const int r0 = it.q0 + t * kSubM;
-      if (!wait_bar(&ctl.fix_empty, (pc & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_arrive_expect_tx(&ctl.fix_full, 2 * kTile);
+      if (Cfg::kFix > 0) {
+        if (!wait_bar(&ctl.fix_empty, (pc & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&ctl.fix_full, 2 * kTile);
 #pragma unroll
-      for (int b = 0; b < Cfg::kBoxes; ++b) {
-        tma_load_3d(sFix + b * kBoxBytes, fix_a, &ctl.fix_full, 64 * b, it.head, r0);
-        tma_load_3d(sFix + kTile + b * kBoxBytes, fix_b, &ctl.fix_full, 64 * b, it.head, r0);
+        for (int b = 0; b < Cfg::kBoxes; ++b) {
+          tma_load_3d(sFix + b * kBoxBytes, fix_a, &ctl.fix_full, 64 * b, it.head, r0);
+          tma_load_3d(sFix + kTile + b * kBoxBytes, fix_b, &ctl.fix_full, 64 * b, it.head, r0);
+        }
+        ++pc;
       }
-      ++pc;
       for (int j = 0; j < it.n_kv && ok; ++j) {
         const int c = it.seg_start + j * kBlockN;
         {
@@ -260,11 +258,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __shared__ BwdCtl ctl;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sP = smem;                  // P^T of the current step (two 64-query boxes)
-  uint8_t* sK = smem + Cfg::kPTileBytes;  // fixed: K_hat then V
-  uint8_t* sV = sK + kTile;
-  uint8_t* sX = sK + 2 * kTile;        // ring of Q_hat
-  uint8_t* sY = sX + NX * kTile;       // ring of dO
+  uint8_t* sK = smem;              // fixed: K_hat then V
+  uint8_t* sV = smem + kTile;
+  uint8_t* sX = smem + 2 * kTile;  // ring of Q_hat
+  uint8_t* sY = sX + NX * kTile;   // ring of dO
   volatile int32_t* abort_flag = &ctl.abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -283,7 +280,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bwd_producer<D, false>(p, ctl, sK, sX, sY, &tmap_k, &tmap_v, &tmap_q, &tmap_do, abort_flag);
   } else if (warp == kBwdMmaWarp) {
     if (lane == 0) {
-      const uint64_t p_desc = smem_desc_sw128(smem_addr(sP), 16, 1024);       // P^T as A of dV
       const uint64_t k_desc = smem_desc_sw128(smem_addr(sK), 16, 1024);
       const uint64_t v_desc = smem_desc_sw128(smem_addr(sV), 16, 1024);
       const uint64_t x_k = smem_desc_sw128(smem_addr(sX), 16, 1024);          // Q_hat as B of S^T
@@ -294,7 +290,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int total_passes, total_steps;
       bwd_counts(p, total_passes, total_steps);
       int pc = 0, g = 0;
-      uint32_t nph = 0, nsf = 0;
+      uint32_t nph = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
         const ItemInfo it = load_item(p.segs, p.work, idx);
@@ -310,19 +306,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!wait_bar(&ctl.y_full[g % NY], (g / NY) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
           issue_qk<D>(tmem + kColDP, v_desc, y_k + (g % NY) * kStep);
-          mma_commit(&ctl.dp_full[0]);
+          mma_commit(&ctl.dp_full);
           for (int j = 0; j < n && ok; ++j) {
             const int gj = g + j, gn = gj + 1;
             const bool more = j + 1 < n;
-            if (more) {
-              // S^T_{j+1} as soon as every softmax warp holds S^T_j
-              if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
-              ++nsf;
-              if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after_sync();
-              issue_qk<D>(tmem + kColS, k_desc, x_k + (gn % NX) * kStep);
-              mma_commit(&ctl.s_full);
-            }
             if (!wait_bar(&ctl.p_ready, nph & 1, abort_flag)) { ok = false; break; }
             tc_fence_after_sync();
             if (j == 0 && pc > 0) {
@@ -330,9 +317,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (!wait_bar(&ctl.acc_empty, (pc - 1) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
             }
-            issue_smem_a<D>(tmem + kColDV, p_desc, y_mn + (gj % NY) * kStep, j > 0);
-            mma_commit(&ctl.p_free);
+            issue_tmem_a<D>(tmem + kColDV, tmem + kColS, y_mn + (gj % NY) * kStep, j > 0);
             if (gj + NY < total_steps) mma_commit(&ctl.y_empty[gj % NY]);
+            if (more) {
+              if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_qk<D>(tmem + kColS, k_desc, x_k + (gn % NX) * kStep);
+              mma_commit(&ctl.s_full);
+            }
             if (!wait_bar(&ctl.ds_ready, nph & 1, abort_flag)) { ok = false; break; }
             ++nph;
             tc_fence_after_sync();
@@ -342,13 +334,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
               issue_qk<D>(tmem + kColDP, v_desc, y_k + (gn % NY) * kStep);
-              mma_commit(&ctl.dp_full[0]);
+              mma_commit(&ctl.dp_full);
             }
           }
           if (!ok) break;
-          // the last S^T of the pass was loaded too: consume its s_free phase
-          if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
-          ++nsf;
           if (pc + 1 < total_passes) mma_commit(&ctl.fix_empty);
           mma_commit(&ctl.acc_ready);
           g += n;
@@ -366,11 +355,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = g4 * 32 + lane;          // key row of the pass
     const uint32_t lane_off = static_cast<uint32_t>(g4 * 32) << 16;
     const uint64_t sl2x2 = f32x2(p.scale_log2, p.scale_log2);
-    // this thread's row of the P^T tile: box h, 128-byte row `row`, 16-byte
-    // chunks at (c ^ (row % 8)) under the 128-byte swizzle
-    uint8_t* p_row = sP + h * kBoxBytes + row * 128;
-    const int swz = row & 7;
-    uint32_t ns = 0, nd = 0, gstep = 0;
+    uint32_t ns = 0, nd = 0;
     int pc = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
@@ -393,59 +378,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool row_in = r0 + row < seg_end;
         float nl0, nl1, d0, d1;
         load_stats(0, nl0, nl1, d0, d1);
-        for (int j = 0; j < it.n_kv; ++j, ++gstep) {
-          if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
-          ++ns;
-          tc_fence_after_sync();
-          uint32_t sr[64];
-          tmem_ld64_sync(tmem + lane_off + kColS + 64 * h, sr);
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl.s_free);
+        for (int j = 0; j < it.n_kv; ++j) {
           // next step's statistics, in flight while this step computes
           float nnl0 = 0.f, nnl1 = 0.f, nd0 = 0.f, nd1 = 0.f;
           if (j + 1 < it.n_kv) load_stats(j + 1, nnl0, nnl1, nd0, nd1);
+          if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
+          ++ns;
+          tc_fence_after_sync();
           uint64_t pp[32];
-          uint32_t pk[32];
+          {
+            uint32_t sr[64];
+            tmem_ld64_sync(tmem + lane_off + kColS + 64 * h, sr);
+            uint32_t pk[32];
 #pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])),
-                                         sl2x2, col_pair(nl0, nl1, c2));
-            float x0, x1;
-            f32x2_split(x, x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            pp[c2] = f32x2(p0, p1);
-            pk[c2] = pack_bf16x2(p0, p1);
+            for (int c2 = 0; c2 < 32; ++c2) {
+              const uint64_t x = fma_f32x2(
+                  f32x2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2x2,
+                  col_pair(nl0, nl1, c2));
+              float x0, x1;
+              f32x2_split(x, x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              pp[c2] = f32x2(p0, p1);
+              pk[c2] = pack_bf16x2(p0, p1);
+            }
+            // P^T over the first 32 columns of this warp's half of S^T
+            tmem_st32_sync(tmem + lane_off + kColS + 64 * h, pk);
           }
-          // P^T_j into shared memory once dV_{j-1} has read P^T_{j-1}
-          if (!warp_wait_bar(&ctl.p_free, (gstep & 1) ^ 1, abort_flag)) { ok = false; break; }
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(p_row + ((c ^ swz) << 4)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          fence_proxy_async_smem();
+          tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl.p_ready);
-          if (!warp_wait_bar(&ctl.dp_full[0], nd & 1, abort_flag)) { ok = false; break; }
+          if (!warp_wait_bar(&ctl.dp_full, nd & 1, abort_flag)) { ok = false; break; }
           ++nd;
           tc_fence_after_sync();
-          // dS in two halves of 32 columns (keeps dP and P in registers together)
+          {
+            uint32_t pk[32];
+            // dS in two halves of 32 columns (keeps dP and P in registers together)
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t dr[32];
-            tmem_ld32_sync(tmem + lane_off + kColDP + 64 * h + 32 * half, dr);
+            for (int half = 0; half < 2; ++half) {
+              uint32_t dr[32];
+              tmem_ld32_sync(tmem + lane_off + kColDP + 64 * h + 32 * half, dr);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c2 = 16 * half + i;
-              const uint64_t ds = mul_f32x2(
-                  pp[c2], sub_f32x2(f32x2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
-                                    col_pair(d0, d1, c2)));
-              float a, b;
-              f32x2_split(ds, a, b);
-              pk[c2] = pack_bf16x2(a, b);
+              for (int i = 0; i < 16; ++i) {
+                const int c2 = 16 * half + i;
+                const uint64_t ds = mul_f32x2(
+                    pp[c2], sub_f32x2(f32x2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
+                                      col_pair(d0, d1, c2)));
+                float a, b;
+                f32x2_split(ds, a, b);
+                pk[c2] = pack_bf16x2(a, b);
+              }
             }
+            tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
           }
-          tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl.ds_ready);
@@ -495,6 +479,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // -------------------------------------------------------------------- dQ ---
 
+// D (+)= A (TMEM, bf16 [128 lanes][K = D], D/2 consecutive columns) *
+// B^T (shared, K-major [N = 128 rows][K = D]): M = 128, N = 128.
+template <int D>
+__device__ __forceinline__ void issue_rows_tmem(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc) {
+  constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, kBlockN, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8,
+           b_desc + static_cast<uint64_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4), kIdesc,
+           kk > 0 ? 1u : 0u);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -503,25 +499,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
   using Cfg = BwdConfig<D, true>;
   constexpr int NX = Cfg::kRingX, NY = Cfg::kRingY, kTile = Cfg::kTileBytes;
-  constexpr uint32_t kColS = 0, kColDQ = 256;
-  constexpr uint32_t kColDP[2] = {128, 384};
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColQ = 384, kColO = 448;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ BwdCtl ctl;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;              // fixed: Q_hat then dO
-  uint8_t* sO = smem + kTile;
-  uint8_t* sX = smem + 2 * kTile;  // ring of K_hat
+  uint8_t* sX = smem;              // ring of K_hat
   uint8_t* sY = sX + NX * kTile;   // ring of V
   volatile int32_t* abort_flag = &ctl.abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  (void)tmap_q;
+  (void)tmap_do;
 
   if (warp == kBwdProducerWarp && lane == 0) {
-    prefetch_tmap(&tmap_q);
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
-    prefetch_tmap(&tmap_do);
   }
   bwd_init<D, true>(ctl, warp);
   const uint32_t tmem = ctl.tmem_base;
@@ -529,11 +522,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (warp == kBwdProducerWarp) {
     if (lane == 0)
-      bwd_producer<D, true>(p, ctl, sQ, sX, sY, &tmap_q, &tmap_do, &tmap_k, &tmap_v, abort_flag);
+      bwd_producer<D, true>(p, ctl, nullptr, sX, sY, nullptr, nullptr, &tmap_k, &tmap_v, abort_flag);
   } else if (warp == kBwdMmaWarp) {
     if (lane == 0) {
-      const uint64_t q_desc = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-      const uint64_t o_desc = smem_desc_sw128(smem_addr(sO), 16, 1024);
       const uint64_t x_k = smem_desc_sw128(smem_addr(sX), 16, 1024);          // K_hat as B of S
       const uint64_t x_mn = smem_desc_sw128(smem_addr(sX), kBoxBytes, 1024);  // K_hat as B of dQ
       const uint64_t y_k = smem_desc_sw128(smem_addr(sY), 16, 1024);          // V as B of dP
@@ -548,51 +539,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int passes = it.b_valid ? 2 : 1;
         for (int t = 0; t < passes && ok; ++t) {
           const int n = it.n_kv;
-          if (!wait_bar(&ctl.fix_full, pc & 1, abort_flag)) { ok = false; break; }
+          // Q_hat and dO of the pass are in TMEM (the previous pass's MMAs
+          // had completed before the softmax warps wrote them)
+          if (!wait_bar(&ctl.q_ready, pc & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
           if (!wait_bar(&ctl.x_full[g % NX], (g / NX) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_qk<D>(tmem + kColS, q_desc, x_k + (g % NX) * kStep);
+          issue_rows_tmem<D>(tmem + kColS, tmem + kColQ, x_k + (g % NX) * kStep);
           mma_commit(&ctl.s_full);
           if (!wait_bar(&ctl.y_full[g % NY], (g / NY) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_qk<D>(tmem + kColDP[0], o_desc, y_k + (g % NY) * kStep);
-          mma_commit(&ctl.dp_full[0]);
+          issue_rows_tmem<D>(tmem + kColDP, tmem + kColO, y_k + (g % NY) * kStep);
+          mma_commit(&ctl.dp_full);
           if (g + NY < total_steps) mma_commit(&ctl.y_empty[g % NY]);
           for (int j = 0; j < n && ok; ++j) {
             const int gj = g + j, gn = gj + 1;
             const bool more = j + 1 < n;
             if (more) {
-              // S_{j+1} and dP_{j+1} as soon as every softmax warp holds S_j
-              // (dP_{j+1} goes to the other buffer; the one it overwrites was
-              // read by dQ_{j-1}, issued before)
+              // S_{j+1} as soon as every softmax warp holds S_j
               if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
               ++nsf;
               if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
-              issue_qk<D>(tmem + kColS, q_desc, x_k + (gn % NX) * kStep);
+              issue_rows_tmem<D>(tmem + kColS, tmem + kColQ, x_k + (gn % NX) * kStep);
               mma_commit(&ctl.s_full);
-              if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after_sync();
-              issue_qk<D>(tmem + kColDP[(j + 1) & 1], o_desc, y_k + (gn % NY) * kStep);
-              mma_commit(&ctl.dp_full[(j + 1) & 1]);
-              if (gn + NY < total_steps) mma_commit(&ctl.y_empty[gn % NY]);
             }
             if (!wait_bar(&ctl.ds_ready, nph & 1, abort_flag)) { ok = false; break; }
             ++nph;
             tc_fence_after_sync();
-            if (j == 0 && pc > 0) {
-              if (!wait_bar(&ctl.acc_empty, (pc - 1) & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after_sync();
-            }
-            issue_tmem_a<D>(tmem + kColDQ, tmem + kColDP[j & 1], x_mn + (gj % NX) * kStep, j > 0);
+            issue_tmem_a<D>(tmem + kColDQ, tmem + kColDP, x_mn + (gj % NX) * kStep, j > 0);
             if (gj + NX < total_steps) mma_commit(&ctl.x_empty[gj % NX]);
+            if (more) {
+              // dP_{j+1} overwrites dS_j only after dQ_j (issued above) has read it
+              if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              issue_rows_tmem<D>(tmem + kColDP, tmem + kColO, y_k + (gn % NY) * kStep);
+              mma_commit(&ctl.dp_full);
+              if (gn + NY < total_steps) mma_commit(&ctl.y_empty[gn % NY]);
+            }
           }
           if (!ok) break;
           // the last S_j was loaded too: consume its s_free phase
           if (!wait_bar(&ctl.s_free, nsf & 1, abort_flag)) { ok = false; break; }
           ++nsf;
-          if (pc + 1 < total_passes) mma_commit(&ctl.fix_empty);
           mma_commit(&ctl.acc_ready);
           g += n;
           ++pc;
@@ -609,7 +598,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = g4 * 32 + lane;  // query row of the pass
     const uint32_t lane_off = static_cast<uint32_t>(g4 * 32) << 16;
     const uint64_t sl2x2 = f32x2(p.scale_log2, p.scale_log2);
-    uint32_t ns = 0, nd[2] = {0, 0};
+    uint32_t ns = 0, nd = 0;
     int pc = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
@@ -620,6 +609,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int r0 = it.q0 + t * kSubM;
         const int q = r0 + row;
         const bool row_in = q < seg_end;
+        // This warp's half of the row's Q_hat and dO into TMEM (columns
+        // [kColQ + D/4 * h, +D/4) and the same for dO); rows past the pack
+        // are zeros. The previous pass's MMAs completed before its epilogue.
+        {
+          constexpr int kV = D / 16;  // 16-byte vectors per half row
+          const size_t base = (static_cast<size_t>(q) * p.heads + it.head) * (D / 8) + kV * h;
+          uint32_t qv[D / 4], ov[D / 4];
+#pragma unroll
+          for (int v = 0; v < kV; ++v) {
+            const uint4 a = q < p.total_tokens ? __ldg(p.q_rows + base + v) : make_uint4(0, 0, 0, 0);
+            const uint4 b = q < p.total_tokens ? __ldg(p.do_rows + base + v) : make_uint4(0, 0, 0, 0);
+            qv[4 * v] = a.x; qv[4 * v + 1] = a.y; qv[4 * v + 2] = a.z; qv[4 * v + 3] = a.w;
+            ov[4 * v] = b.x; ov[4 * v + 1] = b.y; ov[4 * v + 2] = b.z; ov[4 * v + 3] = b.w;
+          }
+          if constexpr (D == 128) {
+            tmem_st32_sync(tmem + lane_off + kColQ + 32 * h, qv);
+            tmem_st32_sync(tmem + lane_off + kColO + 32 * h, ov);
+          } else {
+            tmem_st16_sync(tmem + lane_off + kColQ + 16 * h, qv);
+            tmem_st16_sync(tmem + lane_off + kColO + 16 * h, ov);
+          }
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.q_ready);
+        }
         const size_t si = static_cast<size_t>(it.head) * p.total_tokens + q;
         const float nl = row_in ? -__ldg(p.lse + si) * kLog2e : 0.0f;
         const float drow = row_in ? __ldg(p.delta + si) : 0.0f;
@@ -648,16 +662,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             f32x2_split(x, x0, x1);
             pp[c2] = f32x2(ex2_approx(x0), ex2_approx(x1));
           }
-          const int b = j & 1;
-          if (!warp_wait_bar(&ctl.dp_full[b], nd[b] & 1, abort_flag)) { ok = false; break; }
-          ++nd[b];
+          if (!warp_wait_bar(&ctl.dp_full, nd & 1, abort_flag)) { ok = false; break; }
+          ++nd;
           tc_fence_after_sync();
           {
             uint32_t pk[32];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
               uint32_t dr[32];
-              tmem_ld32_sync(tmem + lane_off + kColDP[b] + 64 * h + 32 * half, dr);
+              tmem_ld32_sync(tmem + lane_off + kColDP + 64 * h + 32 * half, dr);
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int c2 = 16 * half + i;
@@ -668,7 +681,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 pk[c2] = pack_bf16x2(a, bb);
               }
             }
-            tmem_st32_sync(tmem + lane_off + kColDP[b] + 64 * h, pk);
+            tmem_st32_sync(tmem + lane_off + kColDP + 64 * h, pk);
           }
           tc_fence_before_sync();
           __syncwarp();

@@ -481,6 +481,8 @@ extern "C" mf_status mf_joint_attn_bwd(
   prm.lse = lse;
   prm.delta = delta;
   prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.q_rows = reinterpret_cast<const uint4*>(ws + bl.fwd.q_hat);
+  prm.do_rows = static_cast<const uint4*>(dout);
   prm.n_work = n_work;
   prm.heads = heads;
   prm.total_tokens = total_tokens;
@@ -513,8 +515,8 @@ extern "C" mf_status mf_joint_attn_bwd(
         g_q_img, g_k_text, g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps,
         frame_dims, static_cast<uint4*>(dq), static_cast<uint4*>(dk), partial);
     const int n_out = 4 * D;
-    mf::dgamma_reduce_kernel<<<(n_out + 255) / 256, 256, 0, s>>>(partial, bl.pro_blocks, n_out,
-                                                                 dgamma);
+    mf::dgamma_reduce_kernel<<<(n_out + 31) / 32, 32 * mf::kReduceWarps, 0, s>>>(
+        partial, bl.pro_blocks, n_out, dgamma);
     return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
   };
   if (head_dim == 128) return run(std::integral_constant<int, 128>{});

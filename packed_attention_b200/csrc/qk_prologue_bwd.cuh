@@ -202,14 +202,29 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_bwd_kernel(
   }
 }
 
-// dgamma[o] = sum over blocks of partial[b][o], in block order.
-__global__ void dgamma_reduce_kernel(const float* __restrict__ partial, int n_blocks, int n_out,
-                                     float* __restrict__ dgamma) {
-  const int o = blockIdx.x * blockDim.x + threadIdx.x;
-  if (o >= n_out) return;
+// dgamma[o] = sum over blocks of partial[b][o]. A CTA of 8 warps owns 32
+// outputs (one per lane); warp w sums the w-th contiguous eighth of the
+// blocks, then the eight partial sums are added in warp order: a fixed
+// order, so the result is the same on every run.
+constexpr int kReduceWarps = 8;
+
+__global__ void __launch_bounds__(32 * kReduceWarps) dgamma_reduce_kernel(
+    const float* __restrict__ partial, int n_blocks, int n_out, float* __restrict__ dgamma) {
+  __shared__ float s_part[kReduceWarps][32];
+  const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
+  const int o = blockIdx.x * 32 + lane;
+  const int per = (n_blocks + kReduceWarps - 1) / kReduceWarps;
+  const int b0 = w * per, b1 = min(n_blocks, b0 + per);
   float s = 0.f;
-  for (int b = 0; b < n_blocks; ++b) s += partial[static_cast<size_t>(b) * n_out + o];
-  dgamma[o] = s;
+  if (o < n_out)
+    for (int b = b0; b < b1; ++b) s += __ldg(partial + static_cast<size_t>(b) * n_out + o);
+  s_part[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && o < n_out) {
+    float t = 0.f;
+    for (int i = 0; i < kReduceWarps; ++i) t += s_part[i][lane];
+    dgamma[o] = t;
+  }
 }
 
 }  // namespace mf
