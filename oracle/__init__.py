@@ -8,9 +8,10 @@ marshals numpy arrays through ctypes.
 
 Parity status: every function is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_pins.py`` (closed forms, invariants and a dense
-brute-force formulation) and, for the gradients of :func:`attn_grad`,
+brute-force formulation), for the gradients of :func:`attn_grad`,
 ``tests/test_oracle_grad_pins.py`` (central finite differences, closed forms
-and invariants); none is "parity unpinned".
+and invariants), and for the sub-layer around the path (``oracle.block``),
+``tests/test_oracle_block_pins.py``; none is "parity unpinned".
 """
 from __future__ import annotations
 

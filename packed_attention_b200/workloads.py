@@ -197,3 +197,44 @@ CFG_PACKS = {
         heads=24, head_dim=128, seed=6,
         notes="four requests (512^2, 1024^2, 4:1, 768x1024), each cond + uncond"),
 }
+
+
+# ------------------------------------------------ the sub-layer around it ---
+
+STREAM_H, STREAM_WQKV, STREAM_BQKV, STREAM_WO, STREAM_BO = 8, 9, 10, 11, 12
+STREAM_SHIFT, STREAM_SCALE, STREAM_GATE = 13, 14, 15
+
+
+def make_block_inputs(w: Workload):
+    """Seeded inputs of the joint-attention sub-layer around the path, for a
+    pack ``w`` with hidden size C = heads * head_dim.
+
+    h: bf16 bits [T, C], N(0, 1). Per modality (0 text, 1 image): w_qkv bf16
+    bits [2, 3C, C] and w_o [2, C, C], N(0, 1/C) so that the products stay
+    O(1); biases b_qkv [2, 3C], b_o [2, C] fp32, 0.02 N(0, 1). Per sample and
+    modality: shift, scale, gate fp32 [n, 2, C], 0.1 N(0, 1). The four
+    QK-norm gammas as in :func:`make_inputs`.
+    """
+    T, C, n = w.total_tokens, w.heads * w.head_dim, len(w.samples)
+
+    def bf16(stream, shape, std):
+        z = synth.normals(w.seed, stream, int(np.prod(shape))).reshape(shape) * std
+        return synth.f64_to_bf16_bits(z)
+
+    def f32(stream, shape, std):
+        z = synth.normals(w.seed, stream, int(np.prod(shape))).reshape(shape) * std
+        return z.astype(np.float32)
+
+    out = {
+        "h": bf16(STREAM_H, (T, C), 1.0),
+        "w_qkv": bf16(STREAM_WQKV, (2, 3 * C, C), 1.0 / np.sqrt(C)),
+        "b_qkv": f32(STREAM_BQKV, (2, 3 * C), 0.02),
+        "w_o": bf16(STREAM_WO, (2, C, C), 1.0 / np.sqrt(C)),
+        "b_o": f32(STREAM_BO, (2, C), 0.02),
+        "shift": f32(STREAM_SHIFT, (n, 2, C), 0.1),
+        "scale": f32(STREAM_SCALE, (n, 2, C), 0.1),
+        "gate": f32(STREAM_GATE, (n, 2, C), 0.1),
+    }
+    g = make_inputs(Workload(w.name, ((0, 1, 1, 1),), w.heads, w.head_dim, w.seed))
+    out.update({k: g[k] for k in ("g_q_text", "g_q_img", "g_k_text", "g_k_img")})
+    return out
