@@ -324,6 +324,46 @@ def training_line(w, key, steps, warmup, peaks, peak_src):
             "tokens_per_s_training": w.total_tokens / ((f_ms + b_ms) / 1e3), "peaks": peak_src}
 
 
+def block_line(w, key, steps, warmup, peaks, peak_src):
+    """Device time of ``mf_attn_block_fwd`` on the pack with hidden size
+    C = heads * head_dim and random weights. FLOPs: the two projections,
+    2*T*C*3C + 2*T*C*C (each row computed once; a 128-row tile holding both
+    modalities is computed twice and that repeat is not credited), plus the
+    attention's 4*H*d*sum L^2."""
+    import torch
+    import packed_attention_b200 as pa
+    from packed_attention_b200.workloads import make_block_inputs
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_block_inputs(w)
+    t = {}
+    for k, v in inp.items():
+        t[k] = (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
+                else torch.from_numpy(np.ascontiguousarray(v))).to(dev)
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=dev)
+    ws = torch.empty(pa.block_workspace_bytes(plan), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(t["h"])
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, warmup)):
+        pa.attn_block_fwd(t["h"], t, t, plan, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        e0.record(stream)
+        pa.attn_block_fwd(t["h"], t, t, plan, out=out, workspace=ws)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if pa.device_error() != 0:
+        raise RuntimeError("kernel reported a device-side error")
+    ms = sorted(e0.elapsed_time(e1) for e0, e1 in evs)[steps // 2]
+    T, C = w.total_tokens, w.heads * w.head_dim
+    gemm = 8.0 * T * C * C
+    return {"workload": w.name, "config": key, "phase": "attention sub-layer", "hidden": C,
+            "median_ms": ms, "gflop_projections": gemm / 1e9, "gflop_attention": w.flops / 1e9,
+            "tflops": (gemm + w.flops) / (ms / 1e3) / 1e12,
+            "tokens_per_s": T / (ms / 1e3), "peaks": peak_src}
+
+
 def report_all(args):
     """One JSON line per workload: device time of both stages, TFLOP/s, tokens/s,
     fraction of the measured peaks (single GPU). Then one line per packed-CFG
@@ -358,6 +398,15 @@ def report_all(args):
                    ("edit_1024sq_rope3d", EXTRA_WORKLOADS["edit_1024sq_rope3d"])]:
         print(json.dumps(training_line(w, key, max(5, args.steps // 5), args.warmup, peaks,
                                        peak_src)), flush=True)
+
+    # The joint-attention sub-layer around the path (adaLN, per-modality QKV
+    # projection with the QK-norm and rotation in its epilogue, attention,
+    # per-modality output projection with gate and residual in its epilogue).
+    from packed_attention_b200.workloads import make_block_inputs
+    for key in (3, 4):
+        w = WORKLOADS[key]
+        print(json.dumps(block_line(w, key, max(5, args.steps // 5), args.warmup, peaks, peak_src)),
+              flush=True)
 
     for name, cp in CFG_PACKS.items():
         w = cp.packed()

@@ -263,6 +263,45 @@ mf_status mf_joint_attn_bwd(const void* q, const void* k, const void* v, const f
                             float* dgamma, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The joint-attention sub-layer around the path, forward: adaLN modulation,
+ * per-modality QKV projection (bias, QK-RMSNorm and rotation fused into the
+ * GEMM's epilogue), the packed joint attention, per-modality output
+ * projection (bias, gate and residual fused into the GEMM's epilogue).
+ * [Mage-Flow paper summary, "Native-Resolution MMDiT (NR-MMDiT)": an MMDiT
+ *  with modality-specific normalization and joint self-attention; "Training
+ *  Infrastructure": adaptive normalization / RoPE / gating fused into CUDA
+ *  kernels.] Readings (the pages give no formula): adaLN as in DiT, text and
+ * image streams with their own parameters as in an MMDiT. For token t of
+ * sample s, modality m (0 text, 1 image), C = heads * head_dim:
+ *   x_t  = LN(h_t) * (1 + scale[s,m]) + shift[s,m]   (LN over C, no affine, eps_ln)
+ *   qkv  = W_qkv[m] x_t + b_qkv[m]; q, k, v = the three C-wide thirds, viewed
+ *          [heads, head_dim]; q and k through the RMSNorm / rotation of
+ *          mf_qk_prologue_3d (eps, frame_dims)
+ *   o    = the packed joint attention (softmax_scale as mf_joint_attn_fwd)
+ *   h'_t = h_t + gate[s,m] * (W_o[m] o_t + b_o[m])
+ * Arguments (device, 16-B aligned unless noted):
+ *   h, h_out            bf16 [T, C]; h_out must not overlap h or the workspace
+ *   shift, scale, gate  fp32 [n_samples, 2, C]
+ *   w_qkv, b_qkv        bf16 [2, 3C, C] (row n of W is output n), fp32 [2, 3C]
+ *   w_o, b_o            bf16 [2, C, C], fp32 [2, C]
+ *   gammas, plan arrays, eps, frame_dims, softmax_scale as mf_joint_attn_fwd_3d
+ *   workspace           >= mf_block_workspace_bytes(T, heads, head_dim), 256-B aligned
+ * MF_ERR_UNSUPPORTED unless head_dim is 64 or 128 and C is a multiple of 128
+ * and at most 4096. Asynchronous on `stream`.
+ */
+size_t mf_block_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim);
+
+mf_status mf_attn_block_fwd(const void* h, const float* shift, const float* scale,
+                            const float* gate, const void* w_qkv, const float* b_qkv,
+                            const void* w_o, const float* b_o, const float* g_q_text,
+                            const float* g_q_img, const float* g_k_text, const float* g_k_img,
+                            const int32_t* cu_seqlens_dev, const mf_segment* segs_dev,
+                            int32_t n_samples, const mf_work_item* work_dev, int32_t n_work,
+                            int32_t total_tokens, int32_t heads, int32_t head_dim, float eps_ln,
+                            float eps, int32_t frame_dims, float softmax_scale, void* h_out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * mf_joint_attn_fwd_static_scratch -- the same forward for callers that
  * cannot allocate device memory at all. The paper has no counterpart to this
  * entry point; it exists for how the library is called, not for the method.

@@ -11,14 +11,16 @@ from ._native import MfError, MF_TILE_M, MF_TILE_N, pack_plan, workspace_bytes  
 __all__ = ["MfError", "MF_TILE_M", "MF_TILE_N", "pack_plan", "workspace_bytes",
            "PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
            "packed_attention", "workspace_views", "device_error", "joint_attention_fwd_lse",
-           "joint_attention_bwd", "joint_attention_autograd", "bwd_workspace_bytes"]
+           "joint_attention_bwd", "joint_attention_autograd", "bwd_workspace_bytes",
+           "attn_block_fwd", "block_workspace_bytes", "block_workspace_views"]
 
 
 def __getattr__(name):
     if name in ("PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
                 "packed_attention", "workspace_views", "device_error", "GAMMA_NAMES",
                 "joint_attention_fwd_lse", "joint_attention_bwd", "joint_attention_autograd",
-                "bwd_workspace_bytes", "JointAttentionFunction"):
+                "bwd_workspace_bytes", "JointAttentionFunction", "attn_block_fwd",
+                "block_workspace_bytes", "block_workspace_views", "BLOCK_PARAMS"):
         from . import api
         return getattr(api, name)
     raise AttributeError(name)

@@ -67,6 +67,9 @@ SIGNATURES = {
     "mf_bwd_workspace_bytes": (SZ, [I32, I32, I32]),
     "mf_joint_attn_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, F32,
                                 I32, F32, P, P, P, P, P, SZ, P]),
+    "mf_block_workspace_bytes": (SZ, [I32, I32, I32]),
+    "mf_attn_block_fwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32,
+                                F32, F32, I32, F32, P, P, SZ, P]),
     "mf_joint_attn_fwd_static_scratch": (I32, [P, P, P, P, P, P, P, P, P, I32, P, I32, I32, I32,
                                                I32, F32, F32, P, P]),
     "mf_selftest_exp2": (I32, [P, P, I32, P]),

@@ -257,3 +257,55 @@ def joint_attention_autograd(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, plan
                              eps: float = 1e-6, softmax_scale: float = 0.0, frame_dims: int = 0):
     return JointAttentionFunction.apply(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, plan, eps,
                                         softmax_scale, frame_dims)
+
+
+# ------------------------------------------------- the sub-layer around it ---
+
+BLOCK_PARAMS = ("shift", "scale", "gate", "w_qkv", "b_qkv", "w_o", "b_o")
+
+
+def block_workspace_bytes(plan: PackedPlan) -> int:
+    return int(lib().mf_block_workspace_bytes(plan.total_tokens, plan.heads, plan.head_dim))
+
+
+def block_workspace_views(ws: torch.Tensor, plan: PackedPlan) -> dict:
+    """Intermediates a finished mf_attn_block_fwd leaves in its workspace:
+    x (adaLN output), v and o (attention output), bf16 [T, C]; q_hat, k_hat."""
+    T, C = plan.total_tokens, plan.heads * plan.head_dim
+    r256 = lambda n: (n + 255) // 256 * 256
+    fwd = plan.workspace_bytes()
+    mat = r256(T * C * 2)
+    x0 = r256(fwd)
+    views = {}
+    for i, name in enumerate(("x", "v", "o")):
+        off = x0 + i * mat
+        views[name] = ws[off:off + T * C * 2].view(torch.bfloat16).view(T, C)
+    views["q_hat"], views["k_hat"] = workspace_views(ws, plan)
+    return views
+
+
+def attn_block_fwd(h, params: dict, gammas: dict, plan: PackedPlan, eps_ln: float = 1e-6,
+                   eps: float = 1e-6, frame_dims: int = 0, softmax_scale: float = 0.0,
+                   out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """The joint-attention sub-layer forward (mf_attn_block_fwd): h bf16 [T, C];
+    params: shift, scale, gate fp32 [n, 2, C], w_qkv bf16 [2, 3C, C], b_qkv
+    fp32 [2, 3C], w_o bf16 [2, C, C], b_o fp32 [2, C]. Returns h' bf16 [T, C]."""
+    C = plan.heads * plan.head_dim
+    if h.dtype != torch.bfloat16 or tuple(h.shape) != (plan.total_tokens, C) or not h.is_contiguous():
+        raise ValueError(f"h must be a contiguous bf16 tensor of shape {(plan.total_tokens, C)}")
+    for name in BLOCK_PARAMS:
+        if not params[name].is_contiguous() or not params[name].is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    gs = _gammas(gammas, plan)
+    if out is None:
+        out = torch.empty_like(h)
+    if workspace is None:
+        workspace = torch.empty(block_workspace_bytes(plan), dtype=torch.uint8, device=h.device)
+    check("mf_attn_block_fwd", lib().mf_attn_block_fwd(
+        _ptr(h), *[_ptr(params[n]) for n in BLOCK_PARAMS], *[_ptr(g) for g in gs],
+        _ptr(plan.cu_seqlens), _ptr(plan.segs), plan.n_samples, _ptr(plan.work), plan.n_work,
+        plan.total_tokens, plan.heads, plan.head_dim, float(eps_ln), float(eps), int(frame_dims),
+        float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+        _stream_handle(stream)))
+    return out

@@ -14,6 +14,7 @@
 
 #include "../../include/mf_attn.h"
 #include "attention_bwd.cuh"
+#include "block.cuh"
 #include "packed_attention.cuh"
 #include "qk_prologue.cuh"
 #include "qk_prologue_bwd.cuh"
@@ -76,6 +77,22 @@ bool encode_thd(CUtensorMap* map, const void* base, int32_t T, int32_t H, int32_
   cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(mf::kSubM)};
   cuuint32_t elem_strides[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Row-major bf16 matrix [rows, cols] as a 2-D tensor (cols, rows) with
+// boxes of 64 columns x box_rows rows and the 128-byte swizzle.
+bool encode_matrix(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                   uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t elem_strides[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                    box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -521,4 +538,168 @@ extern "C" mf_status mf_joint_attn_bwd(
   };
   if (head_dim == 128) return run(std::integral_constant<int, 128>{});
   return run(std::integral_constant<int, 64>{});
+}
+
+// --------------------------------------------------------- the sub-layer ---
+
+namespace {
+
+struct BlockLayout {
+  WorkspaceLayout fwd;
+  size_t x, v, o, rope, mods, total;
+  int n_mtiles;
+};
+
+bool block_layout(int32_t total_tokens, int32_t heads, int32_t head_dim, BlockLayout* b) {
+  if (!layout(total_tokens, heads, head_dim, &b->fwd)) return false;
+  const size_t C = static_cast<size_t>(heads) * head_dim;
+  const size_t mat = round_up(static_cast<size_t>(total_tokens) * C * 2, kAlign);
+  b->n_mtiles = (total_tokens + mf::kGemmM - 1) / mf::kGemmM;
+  b->x = round_up(b->fwd.total, kAlign);
+  b->v = b->x + mat;
+  b->o = b->v + mat;
+  b->rope = b->o + mat;
+  b->mods = b->rope + round_up(static_cast<size_t>(total_tokens) * (head_dim / 2) * 8, kAlign);
+  b->total = b->mods + round_up(static_cast<size_t>(b->n_mtiles), kAlign);
+  return true;
+}
+
+template <class Epi>
+bool prepare_gemm_kernel() {
+  static std::once_flag once[kMaxDevices];
+  static bool ok[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::call_once(once[dev], [dev] {
+    ok[dev] = cudaFuncSetAttribute(mf::gemm_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   mf::kGemmSmemBytes) == cudaSuccess;
+  });
+  return ok[dev];
+}
+
+}  // namespace
+
+extern "C" size_t mf_block_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim) {
+  BlockLayout b;
+  return block_layout(total_tokens, heads, head_dim, &b) ? b.total : 0;
+}
+
+extern "C" mf_status mf_attn_block_fwd(
+    const void* h, const float* shift, const float* scale, const float* gate, const void* w_qkv,
+    const float* b_qkv, const void* w_o, const float* b_o, const float* g_q_text,
+    const float* g_q_img, const float* g_k_text, const float* g_k_img,
+    const int32_t* cu_seqlens_dev, const mf_segment* segs_dev, int32_t n_samples,
+    const mf_work_item* work_dev, int32_t n_work, int32_t total_tokens, int32_t heads,
+    int32_t head_dim, float eps_ln, float eps, int32_t frame_dims, float softmax_scale,
+    void* h_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (head_dim != 64 && head_dim != 128) return MF_ERR_UNSUPPORTED;
+  const int64_t C = static_cast<int64_t>(heads) * head_dim;
+  if (heads < 1 || C % 128 != 0 || C > mf::kAdalnMaxC) return MF_ERR_UNSUPPORTED;
+  BlockLayout bl;
+  if (!block_layout(total_tokens, heads, head_dim, &bl) || n_samples < 1 || n_work < 1)
+    return MF_ERR_INVALID_ARG;
+  if (!h || !shift || !scale || !gate || !w_qkv || !b_qkv || !w_o || !b_o || !g_q_text ||
+      !g_q_img || !g_k_text || !g_k_img || !cu_seqlens_dev || !segs_dev || !work_dev || !h_out ||
+      !workspace)
+    return MF_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps) || !(eps_ln >= 0.0f) || !std::isfinite(eps_ln) ||
+      !std::isfinite(softmax_scale))
+    return MF_ERR_INVALID_ARG;
+  if (frame_dims < 0 || frame_dims % 4 != 0 || frame_dims > head_dim - 4) return MF_ERR_INVALID_ARG;
+  const void* al16[] = {h, shift, scale, gate, w_qkv, b_qkv, w_o, b_o, h_out};
+  for (const void* ptr : al16)
+    if (!aligned16(ptr)) return MF_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return MF_ERR_ALIGNMENT;
+  if (workspace_bytes < bl.total) return MF_ERR_WORKSPACE;
+  const size_t hb = static_cast<size_t>(total_tokens) * C * 2;
+  if (overlaps(h_out, hb, h, hb) || overlaps(h_out, hb, workspace, bl.total))
+    return MF_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto* x = reinterpret_cast<__nv_bfloat16*>(ws + bl.x);
+  auto* vb = reinterpret_cast<__nv_bfloat16*>(ws + bl.v);
+  auto* ob = reinterpret_cast<__nv_bfloat16*>(ws + bl.o);
+  auto* rope = reinterpret_cast<float2*>(ws + bl.rope);
+  auto* mods = ws + bl.mods;
+  const int sms = sm_count();
+  if (sms <= 0) return MF_ERR_CUDA;
+
+  CUtensorMap ta_x, tb_qkv, ta_o, tb_o;
+  if (!encode_matrix(&ta_x, x, total_tokens, C, mf::kGemmM) ||
+      !encode_matrix(&tb_qkv, w_qkv, 2 * 3 * C, C, mf::kGemmN) ||
+      !encode_matrix(&ta_o, ob, total_tokens, C, mf::kGemmM) ||
+      !encode_matrix(&tb_o, w_o, 2 * C, C, mf::kGemmN))
+    return MF_ERR_CUDA;
+
+  mf::GemmParams gp{};
+  gp.rows = total_tokens;
+  gp.k = static_cast<int>(C);
+  gp.n_mtiles = bl.n_mtiles;
+  gp.tile_mods = mods;
+  gp.cu_seqlens = cu_seqlens_dev;
+  gp.segs = segs_dev;
+  gp.n_samples = n_samples;
+  gp.heads = heads;
+  gp.C = static_cast<int>(C);
+  gp.eps = eps;
+  gp.gammas[0] = g_q_text;
+  gp.gammas[1] = g_q_img;
+  gp.gammas[2] = g_k_text;
+  gp.gammas[3] = g_k_img;
+  gp.rope = rope;
+  gp.q_hat = reinterpret_cast<__nv_bfloat16*>(ws + bl.fwd.q_hat);
+  gp.k_hat = reinterpret_cast<__nv_bfloat16*>(ws + bl.fwd.k_hat);
+  gp.v = vb;
+  gp.h = static_cast<const __nv_bfloat16*>(h);
+  gp.gate = gate;
+  gp.h_out = static_cast<__nv_bfloat16*>(h_out);
+
+  mf::tile_mods_kernel<<<bl.n_mtiles, mf::kGemmM, 0, s>>>(cu_seqlens_dev, segs_dev, n_samples,
+                                                          total_tokens, mods);
+  const int pairs = total_tokens * (head_dim / 2);
+  if (head_dim == 128)
+    mf::rope_table_kernel<128><<<(pairs + 255) / 256, 256, 0, s>>>(cu_seqlens_dev, segs_dev,
+                                                                   n_samples, total_tokens,
+                                                                   frame_dims, rope);
+  else
+    mf::rope_table_kernel<64><<<(pairs + 255) / 256, 256, 0, s>>>(cu_seqlens_dev, segs_dev,
+                                                                  n_samples, total_tokens,
+                                                                  frame_dims, rope);
+  mf::adaln_kernel<<<(total_tokens + 7) / 8, 256, 0, s>>>(
+      static_cast<const uint4*>(h), shift, scale, cu_seqlens_dev, segs_dev, n_samples,
+      total_tokens, static_cast<int>(C), eps_ln, reinterpret_cast<uint4*>(x));
+
+  // QKV projection with the QK-RMSNorm and rotation in its epilogue
+  mf::GemmParams g1 = gp;
+  g1.n_out = static_cast<int>(3 * C);
+  g1.n_ntiles = static_cast<int>((3 * C + mf::kGemmN - 1) / mf::kGemmN);
+  g1.bias = b_qkv;
+  const int items1 = g1.n_mtiles * g1.n_ntiles;
+  const unsigned grid1 = static_cast<unsigned>(items1 < sms ? items1 : sms);
+  if (head_dim == 128) {
+    if (!prepare_gemm_kernel<mf::EpiQkv<128>>()) return MF_ERR_CUDA;
+    mf::gemm_kernel<mf::EpiQkv<128>><<<grid1, mf::kGemmThreads, mf::kGemmSmemBytes, s>>>(ta_x, tb_qkv, g1);
+  } else {
+    if (!prepare_gemm_kernel<mf::EpiQkv<64>>()) return MF_ERR_CUDA;
+    mf::gemm_kernel<mf::EpiQkv<64>><<<grid1, mf::kGemmThreads, mf::kGemmSmemBytes, s>>>(ta_x, tb_qkv, g1);
+  }
+  if (cudaGetLastError() != cudaSuccess) return MF_ERR_CUDA;
+
+  // the packed joint attention of q_hat, k_hat (already in the workspace) and v
+  mf_status st = packed_attention_impl(vb, segs_dev, n_samples, work_dev, n_work, total_tokens,
+                                       heads, head_dim, softmax_scale, ob, nullptr, workspace,
+                                       bl.fwd.total, stream);
+  if (st != MF_OK) return st;
+
+  // output projection with bias, gate and residual in its epilogue
+  mf::GemmParams g2 = gp;
+  g2.n_out = static_cast<int>(C);
+  g2.n_ntiles = static_cast<int>((C + mf::kGemmN - 1) / mf::kGemmN);
+  g2.bias = b_o;
+  const int items2 = g2.n_mtiles * g2.n_ntiles;
+  const unsigned grid2 = static_cast<unsigned>(items2 < sms ? items2 : sms);
+  if (!prepare_gemm_kernel<mf::EpiOut>()) return MF_ERR_CUDA;
+  mf::gemm_kernel<mf::EpiOut><<<grid2, mf::kGemmThreads, mf::kGemmSmemBytes, s>>>(ta_o, tb_o, g2);
+  return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
 }
