@@ -8,8 +8,9 @@ GEMM epilogue (Mage-Flow paper summary, "Native-Resolution MMDiT (NR-MMDiT)",
 Tolerances: x, v are one bf16 rounding of fp32 arithmetic on bf16 inputs
 (2^-8 relative, with slack for the fp32 reduction over C); o carries the
 attention's error (rel-RMS 5e-3, the forward's bound); h' = h + gate * y is
-rounded to bf16 once, so its error is half an ulp of h' plus the error of
-gate * y, which is bounded relative to the update's RMS.
+rounded to bf16 once, so its error is within one ulp of h' (half an ulp,
+doubled where the rounding crosses a power of two) plus the error of gate * y,
+which is bounded relative to the update's RMS.
 """
 import json
 import os
@@ -95,9 +96,10 @@ def test_block_matches_oracle(cuda_device, w, frame_dims):
     report(f"{w.name}_F{fd}", errs)
     assert errs["x"][0] < 4e-3 and errs["v"][0] < 6e-3, errs
     assert errs["o"][0] < 1e-2, errs
-    # h' is rounded once to bf16: within half an ulp of h' plus 2% of the update
-    half_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref["h_out"]), 1e-30))) - 8)
-    assert np.all(np.abs(d) <= half_ulp + 0.02 * np.sqrt(np.mean(upd ** 2)) + 1e-6), errs
+    # h' is rounded once to bf16: within one ulp of h' (half an ulp, doubled
+    # where the rounding crosses a power of two) plus 2% of the update's RMS
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref["h_out"]), 1e-30))) - 7)
+    assert np.all(np.abs(d) <= ulp + 0.02 * np.sqrt(np.mean(upd ** 2)) + 1e-6), errs
 
 
 def test_block_gate_zero_returns_h(cuda_device):
@@ -142,5 +144,5 @@ def test_block_full_size_sampled(cuda_device):
     y = np.stack([o[i] @ p["w_o"][mod[t]].T + p["b_o"][mod[t]] for i, t in enumerate(rows)])
     ref = h[rows] + p["gate"][sid[rows], mod[rows]] * y
     d = bf16_to_f64(out)[rows] - ref
-    half_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
-    assert np.all(np.abs(d) <= half_ulp + 1e-3), float(np.max(np.abs(d)))
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    assert np.all(np.abs(d) <= ulp + 1e-3), float(np.max(np.abs(d)))
