@@ -96,10 +96,13 @@ def test_block_matches_oracle(cuda_device, w, frame_dims):
     report(f"{w.name}_F{fd}", errs)
     assert errs["x"][0] < 4e-3 and errs["v"][0] < 6e-3, errs
     assert errs["o"][0] < 1e-2, errs
-    # h' is rounded once to bf16: within one ulp of h' (half an ulp, doubled
-    # where the rounding crosses a power of two) plus 2% of the update's RMS
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref["h_out"]), 1e-30))) - 7)
-    assert np.all(np.abs(d) <= ulp + 0.02 * np.sqrt(np.mean(upd ** 2)) + 1e-6), errs
+    # h' is rounded once to bf16: within one ulp of the larger of the two
+    # values (half an ulp, doubled where the rounding crosses a power of two)
+    # plus 2% of the update's RMS
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.maximum(np.abs(ref["h_out"]), np.abs(got)),
+                                              1e-30))) - 7)
+    bad = np.abs(d) > ulp + 0.02 * np.sqrt(np.mean(upd ** 2)) + 1e-6
+    assert not bad.any(), (int(bad.sum()), errs, ref["h_out"][bad][:4], got[bad][:4])
 
 
 def test_block_gate_zero_returns_h(cuda_device):
@@ -144,5 +147,6 @@ def test_block_full_size_sampled(cuda_device):
     y = np.stack([o[i] @ p["w_o"][mod[t]].T + p["b_o"][mod[t]] for i, t in enumerate(rows)])
     ref = h[rows] + p["gate"][sid[rows], mod[rows]] * y
     d = bf16_to_f64(out)[rows] - ref
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    got = bf16_to_f64(out)[rows]
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.maximum(np.abs(ref), np.abs(got)), 1e-30))) - 7)
     assert np.all(np.abs(d) <= ulp + 1e-3), float(np.max(np.abs(d)))
