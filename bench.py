@@ -55,6 +55,9 @@ def parse_args():
                     help="workload index 0-4 (default 4), or 'all' for one report line per "
                          "workload (timing only, no e2e / CPU baseline)")
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--block", action="store_true",
+                    help="time the joint-attention sub-layer around the path (adaLN, "
+                         "projections, attention, gate) of the chosen workload on one GPU")
     ap.add_argument("--train", action="store_true",
                     help="time the training pass (forward with log-normaliser + backward) of "
                          "the chosen workload on one GPU and print one JSON line")
@@ -438,6 +441,13 @@ def main():
         report_all(args)
         return
     w = WORKLOADS[int(args.config)]
+    if args.block:
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        peaks, peak_src = load_peaks()
+        print(json.dumps(block_line(w, int(args.config), args.steps, args.warmup, peaks, peak_src)),
+              flush=True)
+        return
     if args.train:
         import torch
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
