@@ -31,7 +31,10 @@
 // there is room, and so do P and dS.
 //
 // dK/dV kernel, per pass: 128 key rows; K_hat and V stay in shared memory and
-// every query step j brings Q_hat_j (3-stage ring) and dO_j (2-stage ring).
+// every query step j brings Q_hat_j and dO_j (2-stage rings each). The
+// per-query statistics of a step (-lse in log2 units, D) go through a small
+// per-warp shared array and are read as broadcast pairs (measured faster than
+// warp shuffles).
 // TMEM columns:
 //   S^T = K_hat Q_hat_j^T [0,128)   P^T (bf16) over [0,32) and [64,96)
 //   dP^T = V dO_j^T     [128,256)   dS^T (bf16) over [128,160) and [192,224)
@@ -73,7 +76,7 @@ struct BwdConfig {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kSubM * D * 2;
   static constexpr int kFix = kDq ? 0 : 2;
-  static constexpr int kRingX = kDq ? 4 : 3;
+  static constexpr int kRingX = kDq ? 4 : 2;
   static constexpr int kRingY = kDq ? 3 : 2;
   static constexpr int kSmemBytes = kTileBytes * (kFix + kRingX + kRingY) + 1024;
 };
@@ -117,12 +120,6 @@ __device__ __forceinline__ void issue_tmem_a(uint32_t d_tmem, uint32_t a_tmem, u
     mma_ts(d_tmem, a_tmem + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
            b_desc + static_cast<uint64_t>(kk * (2048 >> 4)), kIdesc,
            (accumulate || kk > 0) ? 1u : 0u);
-}
-
-// Column c (0..63) of a warp's half: value held by lane c / 2, low or high
-// element (the layout in which the softmax warps hold per-column statistics).
-__device__ __forceinline__ uint64_t col_pair(float lo, float hi, int c2) {
-  return f32x2(__shfl_sync(0xffffffffu, lo, c2), __shfl_sync(0xffffffffu, hi, c2));
 }
 
 template <int D, bool kDq>
@@ -256,6 +253,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ BwdCtl ctl;
+  __shared__ __align__(16) float s_stat[8][2][64];  // per softmax warp: -lse2, D of 64 queries
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;              // fixed: K_hat then V
@@ -382,6 +380,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // next step's statistics, in flight while this step computes
           float nnl0 = 0.f, nnl1 = 0.f, nd0 = 0.f, nd1 = 0.f;
           if (j + 1 < it.n_kv) load_stats(j + 1, nnl0, nnl1, nd0, nd1);
+          float* st_l = s_stat[warp][0];
+          float* st_d = s_stat[warp][1];
+          __syncwarp();
+          st_l[2 * lane] = nl0; st_l[2 * lane + 1] = nl1;
+          st_d[2 * lane] = d0; st_d[2 * lane + 1] = d1;
+          __syncwarp();
           if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
           ++ns;
           tc_fence_after_sync();
@@ -392,9 +396,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             uint32_t pk[32];
 #pragma unroll
             for (int c2 = 0; c2 < 32; ++c2) {
+              const float2 nl = reinterpret_cast<const float2*>(st_l)[c2];
               const uint64_t x = fma_f32x2(
                   f32x2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2x2,
-                  col_pair(nl0, nl1, c2));
+                  f32x2(nl.x, nl.y));
               float x0, x1;
               f32x2_split(x, x0, x1);
               const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
@@ -420,9 +425,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int c2 = 16 * half + i;
+                const float2 dd = reinterpret_cast<const float2*>(st_d)[c2];
                 const uint64_t ds = mul_f32x2(
                     pp[c2], sub_f32x2(f32x2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
-                                      col_pair(d0, d1, c2)));
+                                      f32x2(dd.x, dd.y)));
                 float a, b;
                 f32x2_split(ds, a, b);
                 pk[c2] = pack_bf16x2(a, b);
