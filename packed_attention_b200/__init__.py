@@ -12,7 +12,7 @@ __all__ = ["MfError", "MF_TILE_M", "MF_TILE_N", "pack_plan", "workspace_bytes",
            "PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
            "packed_attention", "workspace_views", "device_error", "joint_attention_fwd_lse",
            "joint_attention_bwd", "joint_attention_autograd", "bwd_workspace_bytes",
-           "attn_block_fwd", "block_workspace_bytes", "block_workspace_views"]
+           "attn_block_fwd", "block_workspace_bytes", "block_workspace_views", "HostPipeline"]
 
 
 def __getattr__(name):
@@ -20,7 +20,8 @@ def __getattr__(name):
                 "packed_attention", "workspace_views", "device_error", "GAMMA_NAMES",
                 "joint_attention_fwd_lse", "joint_attention_bwd", "joint_attention_autograd",
                 "bwd_workspace_bytes", "JointAttentionFunction", "attn_block_fwd",
-                "block_workspace_bytes", "block_workspace_views", "BLOCK_PARAMS"):
+                "block_workspace_bytes", "block_workspace_views", "BLOCK_PARAMS",
+                "HostPipeline"):
         from . import api
         return getattr(api, name)
     raise AttributeError(name)

@@ -309,3 +309,69 @@ def attn_block_fwd(h, params: dict, gammas: dict, plan: PackedPlan, eps_ln: floa
         float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
         _stream_handle(stream)))
     return out
+
+
+# ------------------------------------------------ streaming host batches ---
+
+class HostPipeline:
+    """The forward over a stream of host-resident batches of one plan, with
+    the copies overlapped: batch n's host-to-device copy runs on one CUDA
+    stream while batch n-1 computes on another and batch n-2's result is read
+    back on a third (PCIe moves both directions at once). Two device buffer
+    sets alternate; a set is reused only after its previous result has been
+    read back. Every batch is still copied in and read out in full.
+
+    ``submit(q, k, v, gammas, out_host)`` takes pinned host tensors (bf16
+    [T, H, d] and the four fp32 [d] gammas) and a pinned ``out_host`` to
+    receive the result; it returns at once. ``synchronize()`` waits for all.
+    """
+
+    def __init__(self, plan: PackedPlan, eps: float = 1e-6, softmax_scale: float = 0.0,
+                 frame_dims: int = 0, depth: int = 2):
+        self.plan, self.eps, self.scale, self.frame_dims = plan, eps, softmax_scale, frame_dims
+        dev = plan.device
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_run = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        shape = (plan.total_tokens, plan.heads, plan.head_dim)
+        self.slots = []
+        for _ in range(depth):
+            b = {n: torch.empty(shape, dtype=torch.bfloat16, device=dev) for n in ("q", "k", "v")}
+            b.update({n: torch.empty(plan.head_dim, dtype=torch.float32, device=dev)
+                      for n in GAMMA_NAMES})
+            b["out"] = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+            b["workspace"] = plan.new_workspace()
+            b["copied"] = torch.cuda.Event()
+            b["computed"] = torch.cuda.Event()
+            b["returned"] = torch.cuda.Event()
+            b["used"] = False
+            self.slots.append(b)
+        self.n = 0
+
+    def submit(self, q, k, v, gammas, out_host):
+        b = self.slots[self.n % len(self.slots)]
+        self.n += 1
+        with torch.cuda.stream(self.s_in):
+            if b["used"]:
+                self.s_in.wait_event(b["returned"])  # its last result has been read back
+            for name, src in (("q", q), ("k", k), ("v", v)):
+                b[name].copy_(src, non_blocking=True)
+            for name in GAMMA_NAMES:
+                b[name].copy_(gammas[name], non_blocking=True)
+            b["copied"].record(self.s_in)
+        with torch.cuda.stream(self.s_run):
+            self.s_run.wait_event(b["copied"])
+            joint_attention(b["q"], b["k"], b["v"], {n: b[n] for n in GAMMA_NAMES}, self.plan,
+                            self.eps, self.scale, out=b["out"], workspace=b["workspace"],
+                            stream=self.s_run, frame_dims=self.frame_dims)
+            b["computed"].record(self.s_run)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(b["computed"])
+            out_host.copy_(b["out"], non_blocking=True)
+            b["returned"].record(self.s_out)
+        b["used"] = True
+        return out_host
+
+    def synchronize(self):
+        for s in (self.s_in, self.s_run, self.s_out):
+            s.synchronize()

@@ -236,3 +236,30 @@ def test_fma_pipe_exp2_accuracy(cuda_device):
                                           4, ctypes.c_void_p(st.cuda_stream)) == 0
     v = y2.cpu().numpy()
     assert np.all(v > 0) and np.all(v < 3e-38) and np.all(np.isfinite(v))
+
+
+def test_host_pipeline_matches_device_path(cuda_device):
+    """HostPipeline (uploads, forwards and read-backs overlapped on three
+    streams) gives every batch exactly what the device call gives it."""
+    w = Workload("pipe", ((30, 12, 12, 1), (5, 7, 9, 2)), heads=3, head_dim=128, seed=40)
+    sets = []
+    for seed in (40, 41, 42):
+        inp = make_inputs(Workload(w.name, w.samples, w.heads, w.head_dim, seed))
+        host = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).pin_memory()
+                for n in ("q", "k", "v")}
+        host.update({n: torch.from_numpy(inp[n]).pin_memory() for n in pa.GAMMA_NAMES})
+        sets.append((inp, host))
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, device=cuda_device)
+    pipe = pa.HostPipeline(plan)
+    outs = []
+    for i in range(7):
+        _, host = sets[i % 3]
+        o = torch.empty((w.total_tokens, w.heads, w.head_dim), dtype=torch.bfloat16, pin_memory=True)
+        outs.append(pipe.submit(host["q"], host["k"], host["v"], host, o))
+    pipe.synchronize()
+    assert pa.device_error() == 0
+    for i, o in enumerate(outs):
+        inp, _ = sets[i % 3]
+        _, _, ref = run_gpu(Workload(w.name, w.samples, w.heads, w.head_dim, 40 + i % 3), inp,
+                            cuda_device)
+        assert torch.equal(o.view(torch.int16), ref.cpu().view(torch.int16)), i
