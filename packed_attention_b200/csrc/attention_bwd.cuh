@@ -24,11 +24,9 @@
 // mbarrier waits throughout. A work item of the forward's list (256 rows of
 // one head of one sample) is done as two passes of 128 rows.
 //
-// Shared-memory bandwidth, not the tensor pipe, is what these kernels must
-// budget: an MMA of 128 x 128 x 16 with both operands in shared memory reads
-// 8 KB in its 64 cycles, the whole 128 B/clk the SM has, while one with A in
-// TMEM reads 4 KB. Operands reused across a pass therefore sit in TMEM where
-// there is room, and so do P and dS.
+// Operands reused across a pass sit in TMEM where there is room, and so do P
+// and dS: an MMA with A in TMEM reads one operand (4 KB for 128 x 128 x 16)
+// from shared memory instead of two.
 //
 // dK/dV kernel, per pass: 128 key rows; K_hat and V stay in shared memory and
 // every query step j brings Q_hat_j and dO_j (2-stage rings each). The
