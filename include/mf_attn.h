@@ -103,8 +103,9 @@ const char* mf_status_string(mf_status status);
  * Outputs (host, caller-owned; each may be NULL to skip it):
  *   cu_seqlens [n_samples + 1]   prefix sums of the sample lengths, int32
  *   segs       [n_samples]       mf_segment per sample
- *   work       [*n_work]         work items ordered longest sample first
- *                                (ties: sample index, then head, then q_tile)
+ *   work       [*n_work]         work items ordered by cost, largest first:
+ *                                sample length x 128-row query sub-tiles in
+ *                                the item (ties: sample index, head, q_tile)
  *   n_work, total_tokens         scalars (may be NULL)
  * Two-call convention: call with work == NULL to learn *n_work, then again
  * with *n_work set to the capacity of `work` (at least the count returned);

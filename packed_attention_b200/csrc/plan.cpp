@@ -6,10 +6,11 @@
 //  packed with their text under a fixed token budget; attention uses
 //  per-sample cumulative offsets. Video overview, 00:04:03: no padding.]
 //
-// The work list holds one item per (sample, head, 256-row query tile). Items
-// are ordered by sample length, longest first, because an item's cost grows
-// with the number of keys it attends over (its sample's length): handing the
-// longest items out first keeps the last wave of the persistent kernel short.
+// The work list holds one item per (sample, head, 256-row query tile). An
+// item's cost grows with the keys it attends over (its sample's length) and
+// with its 128-row query sub-tiles (the last tile of a sample may hold only
+// one). Items are ordered by that cost, largest first: handing the expensive
+// items out first keeps the last wave of the persistent kernel short.
 
 #include <algorithm>
 #include <cstdint>
@@ -78,16 +79,20 @@ extern "C" mf_status mf_pack_plan(int32_t n_samples, const int32_t* n_text,
     return MF_ERR_INVALID_ARG;
   }
   if (work) {
-    std::vector<int32_t> order(static_cast<size_t>(n_samples));
-    for (int32_t i = 0; i < n_samples; ++i) order[i] = i;
-    std::stable_sort(order.begin(), order.end(),
-                     [&](int32_t a, int32_t b) { return seg[a].len > seg[b].len; });
     int64_t w = 0;
-    for (int32_t si : order) {
+    for (int32_t si = 0; si < n_samples; ++si) {
       const int32_t tiles = (seg[si].len + MF_TILE_M - 1) / MF_TILE_M;
       for (int32_t h = 0; h < heads; ++h)
         for (int32_t qt = 0; qt < tiles; ++qt) work[w++] = mf_work_item{si, h, qt, seg[si].len};
     }
+    // cost: keys x query sub-tiles (a last tile of at most half the rows has one)
+    auto cost = [&](const mf_work_item& it) {
+      const int64_t rows = std::min<int64_t>(MF_TILE_M, seg[it.seg].len - int64_t{it.q_tile} * MF_TILE_M);
+      return int64_t{it.kv_len} * (rows > MF_TILE_M / 2 ? 2 : 1);
+    };
+    std::stable_sort(work, work + w, [&](const mf_work_item& a, const mf_work_item& b) {
+      return cost(a) > cost(b);
+    });
   }
   return MF_OK;
 }

@@ -80,9 +80,14 @@ def test_plan_work_list(lib, cfg, n_work):
             for t in range((lens[s] + pa.MF_TILE_M - 1) // pa.MF_TILE_M)}
     got = {tuple(x) for x in work[:, :3].tolist()}
     assert got == want and len(got) == n_work
-    # kv_len is the segment length; longest first, ties by sample index then head, q_tile
+    # kv_len is the segment length; ordered by cost = length x query sub-tiles
+    # (a last tile of at most 128 rows has one), largest first; ties by
+    # sample index, then head, then q_tile
     assert np.array_equal(work[:, 3], lens[work[:, 0]])
-    keys = [(-int(L), int(s), int(h), int(t)) for s, h, t, L in work.tolist()]
+    def cost(s, t, L):
+        rows = min(pa.MF_TILE_M, L - t * pa.MF_TILE_M)
+        return L * (2 if rows > pa.MF_TILE_M // 2 else 1)
+    keys = [(-cost(s, t, L), int(s), int(h), int(t)) for s, h, t, L in work.tolist()]
     assert keys == sorted(keys)
 
 
