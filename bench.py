@@ -272,6 +272,27 @@ def _median_step_ms(runs, steps, warmup):
     return total, pro, att
 
 
+def _prologue_ms_flushed(run, steps):
+    """Median prologue time (ms) with L2 flushed before each launch: a
+    256 MB buffer (twice the 126 MB L2) is written between launches, outside
+    the timed interval."""
+    import torch
+    import packed_attention_b200 as pa
+    t, plan, ws, out, eps, frame_dims = run
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=t["q"].device)
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pa.qk_prologue(t["q"], t["k"], t, plan, ws, eps=eps, frame_dims=frame_dims)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return sorted(times)[len(times) // 2]
+
+
 def training_line(w, key, steps, warmup, peaks, peak_src):
     """Device time of one training pass over the pack: the forward with its
     log-normaliser (``mf_joint_attn_fwd_lse``) and the backward
@@ -384,7 +405,9 @@ def report_all(args):
         return (t, plan, plan.new_workspace(), torch.empty_like(t["q"]), w.eps, w.rope_frame_dims)
 
     for cfg, w in list(WORKLOADS.items()) + list(EXTRA_WORKLOADS.items()):
-        _, pro, att = _median_step_ms([prepare(w, make_inputs(w))], args.steps, args.warmup)
+        run = prepare(w, make_inputs(w))
+        _, pro, att = _median_step_ms([run], args.steps, args.warmup)
+        pro_flushed = _prologue_ms_flushed(run, 20)
         T, H, d = w.total_tokens, w.heads, w.head_dim
         print(json.dumps({
             "workload": w.name, "config": cfg, "total_tokens": T, "heads": H, "head_dim": d,
@@ -394,6 +417,7 @@ def report_all(args):
             "frac_sustained_peak_attention": w.flops / (att / 1e3) / 1e12 / sustained,
             "tokens_per_s": T / ((pro + att) / 1e3),
             "prologue_gbs": 8 * T * H * d / (pro / 1e3) / 1e9,
+            "prologue_gbs_l2_flushed": 8 * T * H * d / (pro_flushed / 1e3) / 1e9,
             "rope_frame_dims": w.rope_frame_dims, "peaks": peak_src}), flush=True)
 
     # Training: forward with the log-normaliser, then the backward.
