@@ -293,7 +293,29 @@ def _prologue_ms_flushed(run, steps):
     return sorted(times)[len(times) // 2]
 
 
-def training_line(w, key, steps, warmup, peaks, peak_src):
+def _oracle_backward_rate(w, inp):
+    """The fp64 oracle's forward + backward (oracle.attn_grad) timed on the
+    host cores on one head of the pack's longest sample: its rate in the
+    backward's FLOP convention (2.5x the forward's 4 * d * L^2)."""
+    import oracle
+    from packed_attention_b200 import synth
+    L = max(w.seg_lens)
+    i = w.seg_lens.index(L)
+    start = sum(w.seg_lens[:i])
+    sl = slice(start, start + L)
+    q, k, v = (synth.bf16_bits_to_f64(inp[n][sl, :1]) for n in ("q", "k", "v"))
+    dout = np.random.default_rng(0).standard_normal(q.shape)
+    gam = {n: inp[n].astype(np.float64) for n in ("g_q_text", "g_q_img", "g_k_text", "g_k_img")}
+    t0 = time.perf_counter()
+    oracle.attn_grad(q, k, v, gam, [w.samples[i]], dout=dout, eps=w.eps,
+                     frame_dims=w.rope_frame_dims)
+    sec = time.perf_counter() - t0
+    flops = 2.5 * 4.0 * w.head_dim * L * L
+    return {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"one head of the {L}-token sample, {sec:.1f} s"}
+
+
+def training_line(w, key, steps, warmup, peaks, peak_src, with_oracle=False):
     """Device time of one training pass over the pack: the forward with its
     log-normaliser (``mf_joint_attn_fwd_lse``) and the backward
     (``mf_joint_attn_bwd``), medians over ``steps``. Backward FLOPs are counted
@@ -340,7 +362,9 @@ def training_line(w, key, steps, warmup, peaks, peak_src):
         raise RuntimeError("kernel reported a device-side error")
     f_ms = sorted(e[0].elapsed_time(e[1]) for e in evs)[steps // 2]
     b_ms = sorted(e[1].elapsed_time(e[2]) for e in evs)[steps // 2]
+    oracle_line = _oracle_backward_rate(w, inp) if with_oracle else None
     return {"workload": w.name, "config": key, "phase": "training",
+            "cpu_oracle_backward": oracle_line,
             "gflop_forward": w.flops / 1e9, "median_ms_forward_lse": f_ms,
             "median_ms_backward": b_ms, "tflops_forward": w.flops / (f_ms / 1e3) / 1e12,
             "tflops_backward": 2.5 * w.flops / (b_ms / 1e3) / 1e12,
@@ -424,7 +448,7 @@ def report_all(args):
     for key, w in [(1, WORKLOADS[1]), (2, WORKLOADS[2]), (3, WORKLOADS[3]), (4, WORKLOADS[4]),
                    ("edit_1024sq_rope3d", EXTRA_WORKLOADS["edit_1024sq_rope3d"])]:
         print(json.dumps(training_line(w, key, max(5, args.steps // 5), args.warmup, peaks,
-                                       peak_src)), flush=True)
+                                       peak_src, with_oracle=key in (1, 3))), flush=True)
 
     # The joint-attention sub-layer around the path (adaLN, per-modality QKV
     # projection with the QK-norm and rotation in its epilogue, attention,
