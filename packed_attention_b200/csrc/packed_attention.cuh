@@ -101,8 +101,12 @@ struct AttnConfig {
   static constexpr int kTileBytes = kSubM * D * 2;  // one 128-row tile of Q, K or V
   // Deep enough that each K/V load is requested a full key step before use.
   static constexpr int kStages = D == 128 ? 4 : 6;
-  static constexpr int kSmemBytes = kTileBytes * (2 + kStages) + 1024;
+  // Per softmax warp: 32 output rows x 64 dims (bf16) staged for coalesced
+  // stores at the end of an item.
+  static constexpr int kStageBytes = 8 * 32 * 128;
+  static constexpr int kSmemBytes = kTileBytes * (2 + kStages) + kStageBytes + 1024;
   static_assert(kStages <= kMaxStages, "ring too deep");
+  static_assert(kSmemBytes <= 226 * 1024, "over the 227 KB of shared memory a CTA may use");
 };
 
 struct AttnParams {
@@ -262,6 +266,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;                // sub-tile a, then sub-tile b
   uint8_t* sKV = smem + 2 * kTile;   // NS stages
+  uint8_t* sOut = sKV + NS * kTile;  // output staging, 4 KB per softmax warp
   volatile int32_t* abort_flag = &ctl.abort;
 
   const int warp = threadIdx.x / 32;
@@ -525,20 +530,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ++no;
       tc_fence_after_sync();
       const int q_row = it.q0 + t * kSubM + row;
-      const bool store = row_in;
       const float inv_l = 1.0f / l;
       // log of the row's softmax normaliser, sum_u exp(s_u * scale), for the
       // backward pass: m and l are in the exp2 domain of s * scale * log2(e).
-      if (p.lse && store)
+      if (p.lse && row_in)
         p.lse[static_cast<size_t>(it.head) * p.total_tokens + q_row] =
             (m + log2f(l)) * 0.6931471805599453f;
-      uint4* dst = reinterpret_cast<uint4*>(p.out) +
-                   (static_cast<size_t>(q_row) * p.heads + it.head) * (D / 8);
+      // O / l in 64-dim halves through this warp's 4 KB of shared memory:
+      // each lane writes its row (128 bytes, 16-byte chunk c at c ^ (row % 8)),
+      // then each store instruction of the warp writes four whole 128-byte row
+      // segments (eight lanes per row) instead of 32 scattered 16-byte pieces.
+      uint8_t* stage = sOut + warp * 4096;
+      const int rr0 = lane >> 3;  // first row this lane stores, then every 4th
+      const int cc = lane & 7;    // 16-byte chunk of the row this lane stores
+      const int row0 = it.q0 + t * kSubM + wl * 32;  // token of the warp's first row
+      const int row_end = it.seg_start + it.seg_len;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32_sync(o_tmem + 32 * c, r);
-        if (store) {
+      for (int half = 0; half < D / 64; ++half) {
+#pragma unroll
+        for (int c32 = 0; c32 < 2; ++c32) {
+          uint32_t r[32];
+          tmem_ld32_sync(o_tmem + 64 * half + 32 * c32, r);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 o;
@@ -546,9 +558,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             o.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * inv_l, __uint_as_float(r[8 * v4 + 3]) * inv_l);
             o.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * inv_l, __uint_as_float(r[8 * v4 + 5]) * inv_l);
             o.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * inv_l, __uint_as_float(r[8 * v4 + 7]) * inv_l);
-            dst[4 * c + v4] = o;
+            const int c = 4 * c32 + v4;
+            *reinterpret_cast<uint4*>(stage + lane * 128 + ((c ^ (lane & 7)) << 4)) = o;
           }
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + rr0;
+          const uint4 o = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((cc ^ (rr & 7)) << 4));
+          const int tok = row0 + rr;
+          if (tok < row_end)
+            reinterpret_cast<uint4*>(p.out)[(static_cast<size_t>(tok) * p.heads + it.head) * (D / 8) +
+                                            8 * half + cc] = o;
+        }
+        __syncwarp();
       }
     }
   }
