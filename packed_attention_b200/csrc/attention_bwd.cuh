@@ -76,8 +76,41 @@ struct BwdConfig {
   static constexpr int kFix = kDq ? 0 : 2;
   static constexpr int kRingX = kDq ? 4 : 2;
   static constexpr int kRingY = kDq ? 3 : 2;
-  static constexpr int kSmemBytes = kTileBytes * (kFix + kRingX + kRingY) + 1024;
+  // dK/dV kernel: 2 KB per softmax warp to stage its output rows.
+  static constexpr int kStageBytes = kDq ? 0 : 8 * 2048;
+  static constexpr int kSmemBytes = kTileBytes * (kFix + kRingX + kRingY) + kStageBytes + 1024;
 };
+
+// 32 rows x 64 bytes of one warp (lane = row) go to rows gbase + r * stride,
+// r < valid_rows, through the warp's 2 KB of shared memory: stage_put places
+// the lane's 16-byte piece c, stage_flush stores, and each of its store
+// instructions writes eight whole 64-byte row segments instead of 32
+// scattered 16-byte pieces. Piece c of row r sits at c ^ ((r / 2) % 4), so
+// that neither side has bank conflicts.
+// (stage is a shared-memory address.)
+__device__ __forceinline__ void stage_put(uint32_t stage, int lane, int c, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                   stage + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void stage_flush(uint32_t stage, int lane, uint8_t* gbase, size_t stride,
+                                            int valid_rows) {
+  __syncwarp();
+  const int q = lane & 3;
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i) {
+    const int rr = 8 * i + (lane >> 2);
+    uint4 o;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+                 : "r"(stage + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4))
+                 : "memory");
+    if (rr < valid_rows) *reinterpret_cast<uint4*>(gbase + rr * stride + q * 16) = o;
+  }
+  __syncwarp();
+}
 
 struct BwdParams {
   const mf_segment* segs;
@@ -258,6 +291,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* sV = smem + kTile;
   uint8_t* sX = smem + 2 * kTile;  // ring of Q_hat
   uint8_t* sY = sX + NX * kTile;   // ring of dO
+  uint8_t* sStage = sY + NY * kTile;  // 2 KB per softmax warp
   volatile int32_t* abort_flag = &ctl.abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -443,33 +477,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // ---- epilogue: dv (bf16) and dk_hat = scale * acc (fp32) rows ----
         if (!warp_wait_bar(&ctl.acc_ready, pc & 1, abort_flag)) { ok = false; break; }
         tc_fence_after_sync();
-        const size_t orow = (static_cast<size_t>(r0 + row) * p.heads + it.head) * D;
+        const int tok0 = r0 + g4 * 32;  // token of this warp's first key row
+        const int valid_rows = seg_end - tok0;
+        const uint32_t stage = smem_addr(sStage) + warp * 2048;
 #pragma unroll 1
         for (int c = 0; c < D / 64; ++c) {
           const int col = h * (D / 2) + 32 * c;
+          const size_t orow0 = (static_cast<size_t>(tok0) * p.heads + it.head) * D + col;
           uint32_t r[32];
           tmem_ld32_sync(tmem + lane_off + kColDV + col, r);
-          if (row_in) {
-            uint4* dst = reinterpret_cast<uint4*>(p.dv + orow + col);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            stage_put(stage, lane, v4,
+                      make_uint4(pack_bf16x2(__uint_as_float(r[8 * v4 + 0]), __uint_as_float(r[8 * v4 + 1])),
+                                 pack_bf16x2(__uint_as_float(r[8 * v4 + 2]), __uint_as_float(r[8 * v4 + 3])),
+                                 pack_bf16x2(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5])),
+                                 pack_bf16x2(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7]))));
+          stage_flush(stage, lane, reinterpret_cast<uint8_t*>(p.dv + orow0),
+                      static_cast<size_t>(p.heads) * D * 2, valid_rows);
+          tmem_ld32_sync(tmem + lane_off + kColDK + col, r);
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r[8 * v4 + 0]), __uint_as_float(r[8 * v4 + 1]));
-              o.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]), __uint_as_float(r[8 * v4 + 3]));
-              o.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5]));
-              o.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7]));
-              dst[v4] = o;
+              const int e = 16 * k2 + 4 * v4;
+              stage_put(stage, lane, v4,
+                        make_uint4(__float_as_uint(__uint_as_float(r[e + 0]) * p.scale),
+                                   __float_as_uint(__uint_as_float(r[e + 1]) * p.scale),
+                                   __float_as_uint(__uint_as_float(r[e + 2]) * p.scale),
+                                   __float_as_uint(__uint_as_float(r[e + 3]) * p.scale)));
             }
-          }
-          tmem_ld32_sync(tmem + lane_off + kColDK + col, r);
-          if (row_in) {
-            float4* dst = reinterpret_cast<float4*>(p.dhat + orow + col);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(r[4 * v + 0]) * p.scale,
-                                   __uint_as_float(r[4 * v + 1]) * p.scale,
-                                   __uint_as_float(r[4 * v + 2]) * p.scale,
-                                   __uint_as_float(r[4 * v + 3]) * p.scale);
+            stage_flush(stage, lane, reinterpret_cast<uint8_t*>(p.dhat + orow0 + 16 * k2),
+                        static_cast<size_t>(p.heads) * D * 4, valid_rows);
           }
         }
         tc_fence_before_sync();
