@@ -75,9 +75,9 @@ struct BwdConfig {
   static constexpr int kTileBytes = kSubM * D * 2;
   static constexpr int kFix = kDq ? 0 : 2;
   static constexpr int kRingX = kDq ? 4 : 2;
-  static constexpr int kRingY = kDq ? 3 : 2;
-  // dK/dV kernel: 2 KB per softmax warp to stage its output rows.
-  static constexpr int kStageBytes = kDq ? 0 : 8 * 2048;
+  static constexpr int kRingY = 2;
+  // 2 KB per softmax warp to stage its output rows.
+  static constexpr int kStageBytes = 8 * 2048;
   static constexpr int kSmemBytes = kTileBytes * (kFix + kRingX + kRingY) + kStageBytes + 1024;
 };
 
@@ -405,7 +405,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       };
       for (int t = 0; t < passes && ok; ++t, ++pc) {
         const int r0 = it.q0 + t * kSubM;
-        const bool row_in = r0 + row < seg_end;
         float nl0, nl1, d0, d1;
         load_stats(0, nl0, nl1, d0, d1);
         for (int j = 0; j < it.n_kv; ++j) {
@@ -550,6 +549,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sX = smem;              // ring of K_hat
   uint8_t* sY = sX + NX * kTile;   // ring of V
+  uint8_t* sStage = sY + NY * kTile;  // 2 KB per softmax warp
   volatile int32_t* abort_flag = &ctl.abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   (void)tmap_q;
@@ -733,20 +733,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!ok) break;
         if (!warp_wait_bar(&ctl.acc_ready, pc & 1, abort_flag)) { ok = false; break; }
         tc_fence_after_sync();
-        const size_t orow = (static_cast<size_t>(q) * p.heads + it.head) * D;
+        const int tok0 = r0 + g4 * 32;  // token of this warp's first query row
+        const int valid_rows = seg_end - tok0;
+        const uint32_t stage = smem_addr(sStage) + warp * 2048;
 #pragma unroll 1
         for (int c = 0; c < D / 64; ++c) {
           const int col = h * (D / 2) + 32 * c;
+          const size_t orow0 = (static_cast<size_t>(tok0) * p.heads + it.head) * D + col;
           uint32_t r[32];
           tmem_ld32_sync(tmem + lane_off + kColDQ + col, r);
-          if (row_in) {
-            float4* dst = reinterpret_cast<float4*>(p.dhat + orow + col);
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(r[4 * v + 0]) * p.scale,
-                                   __uint_as_float(r[4 * v + 1]) * p.scale,
-                                   __uint_as_float(r[4 * v + 2]) * p.scale,
-                                   __uint_as_float(r[4 * v + 3]) * p.scale);
+          for (int k2 = 0; k2 < 2; ++k2) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const int e = 16 * k2 + 4 * v4;
+              stage_put(stage, lane, v4,
+                        make_uint4(__float_as_uint(__uint_as_float(r[e + 0]) * p.scale),
+                                   __float_as_uint(__uint_as_float(r[e + 1]) * p.scale),
+                                   __float_as_uint(__uint_as_float(r[e + 2]) * p.scale),
+                                   __float_as_uint(__uint_as_float(r[e + 3]) * p.scale)));
+            }
+            stage_flush(stage, lane, reinterpret_cast<uint8_t*>(p.dhat + orow0 + 16 * k2),
+                        static_cast<size_t>(p.heads) * D * 4, valid_rows);
           }
         }
         tc_fence_before_sync();
