@@ -382,7 +382,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------- softmax and epilogue ---
     const int g4 = warp & 3, h = warp >> 2;  // TMEM lane quarter, column half
-    const int row = g4 * 32 + lane;          // key row of the pass
     const uint32_t lane_off = static_cast<uint32_t>(g4 * 32) << 16;
     const uint64_t sl2x2 = f32x2(p.scale_log2, p.scale_log2);
     uint32_t ns = 0, nd = 0;
