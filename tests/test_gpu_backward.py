@@ -102,6 +102,12 @@ SMALL = [
     Workload("frames3d_d128", ((30, 9, 11, 2), (3, 7, 5, 3)), heads=2, head_dim=128, seed=14,
              rope_frame_dims=16),
     Workload("frames3d_d64", ((0, 12, 12, 2),), heads=2, head_dim=64, seed=15, rope_frame_dims=8),
+    # sample ends at and one past the 32-row boundaries of a warp's output rows
+    Workload("warp_edges", ((31, 1, 1, 1), (32, 1, 1, 1), (62, 1, 1, 1), (63, 1, 1, 1),
+                            (95, 1, 1, 1), (0, 1, 97, 1), (0, 8, 20, 1)), heads=2, head_dim=128,
+             seed=16),
+    Workload("warp_edges_d64", ((31, 1, 1, 1), (0, 1, 33, 1), (63, 1, 1, 1), (0, 5, 19, 1)),
+             heads=3, head_dim=64, seed=17),
 ]
 
 

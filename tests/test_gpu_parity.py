@@ -112,6 +112,13 @@ SMALL_PACKS = [
                                            (0, 1, 129, 1), (1, 16, 16, 1), (0, 1, 257, 1)),
                             heads=2, head_dim=128, seed=13)),
     ("config2_shapes_h1", WORKLOADS[2].with_heads(1)),
+    # sample ends at and one past the 32-row boundaries of a softmax warp's
+    # output rows (the epilogue stores a warp's rows together)
+    ("warp_edges", Workload("warp_edges", ((31, 1, 1, 1), (32, 1, 1, 1), (62, 1, 1, 1),
+                                           (63, 1, 1, 1), (95, 1, 1, 1), (0, 1, 97, 1),
+                                           (0, 8, 20, 1)), heads=2, head_dim=128, seed=16)),
+    ("warp_edges_d64", Workload("warp_edges_d64", ((31, 1, 1, 1), (0, 1, 33, 1), (63, 1, 1, 1),
+                                                   (0, 5, 19, 1)), heads=3, head_dim=64, seed=17)),
 ]
 
 
