@@ -123,6 +123,30 @@ mf_status mf_pack_plan(int32_t n_samples, const int32_t* n_text, const int32_t* 
                        int32_t* total_tokens);
 
 /*
+ * mf_schedule_work -- host only; assigns a work list to n_ctas persistent
+ * CTAs ahead of time, longest processing time first: items in decreasing
+ * cost (key steps x 20 with two query sub-tiles, x 19 with one: a lone
+ * sub-tile's step is the softmax -> PV -> next-S chain by itself, about 95 %
+ * of a two-sub-tile step; ties keep the input order), each to the CTA with
+ * the least work so far (lowest index on ties). The result is laid out
+ * for the kernels' traversal, in which CTA c takes positions c, c + n_ctas,
+ * c + 2 n_ctas, ...: position r * n_ctas + c holds CTA c's r-th item, and a
+ * CTA with fewer items than the busiest is padded with {0, 0, -1, 0}
+ * entries (q_tile < 0), which every kernel skips. Launched on any other
+ * number of CTAs the list stays correct (every item runs once), only the
+ * balance is lost; the library launches min(n_work, SM count) CTAs.
+ *   work, n_work   a work list from mf_pack_plan (host)
+ *   n_ctas         CTAs to balance over (>= 1; capped at n_work)
+ *   sched          [*n_sched] output (host, caller-owned), or NULL
+ *   n_sched        with sched == NULL receives the length; otherwise the
+ *                  capacity of sched on entry and the length written on exit
+ * Errors: MF_ERR_INVALID_ARG for NULL arguments, n_work < 1, n_ctas < 1,
+ * an input entry with q_tile < 0, or too small a capacity.
+ */
+mf_status mf_schedule_work(const mf_work_item* work, int32_t n_work, int32_t n_ctas,
+                           mf_work_item* sched, int32_t* n_sched);
+
+/*
  * Bytes of device workspace mf_joint_attn_fwd needs: the normalised, rotated
  * q_hat and k_hat ([T, H, d] bf16 each) plus a small control block.
  * Returns 0 for invalid sizes.

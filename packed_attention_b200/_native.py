@@ -54,6 +54,7 @@ SIGNATURES = {
     "mf_abi_version": (I32, []),
     "mf_status_string": (ctypes.c_char_p, [I32]),
     "mf_pack_plan": (I32, [I32, P, P, P, P, I32, I32, I64, P, P, P, P, P]),
+    "mf_schedule_work": (I32, [P, I32, I32, P, P]),
     "mf_workspace_bytes": (SZ, [I32, I32, I32]),
     "mf_qk_prologue": (I32, [P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, P, SZ, P]),
     "mf_qk_prologue_3d": (I32, [P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, I32, P, SZ, P]),
@@ -126,6 +127,20 @@ def pack_plan(samples, heads: int, head_dim: int, token_budget: int = 0):
                                          ctypes.byref(total)))
     return {"cu_seqlens": cu, "segs": segs, "work": work, "total_tokens": int(total.value),
             "n_samples": n, "heads": heads, "head_dim": head_dim}
+
+
+def schedule_work(work, n_ctas: int):
+    """``work`` ([n, 4] int32, from pack_plan) laid out for ``n_ctas`` CTAs by
+    ``mf_schedule_work``: [rounds * n_ctas, 4], padding rows have q_tile -1."""
+    work = np.ascontiguousarray(work, dtype=np.int32).reshape(-1, 4)
+    n_sched = ctypes.c_int32(0)
+    L = lib()
+    check("mf_schedule_work", L.mf_schedule_work(work.ctypes.data_as(P), len(work), n_ctas, None,
+                                                 ctypes.byref(n_sched)))
+    sched = np.zeros((n_sched.value, 4), dtype=np.int32)
+    check("mf_schedule_work", L.mf_schedule_work(work.ctypes.data_as(P), len(work), n_ctas,
+                                                 sched.ctypes.data_as(P), ctypes.byref(n_sched)))
+    return sched[:n_sched.value]
 
 
 def workspace_bytes(total_tokens: int, heads: int, head_dim: int) -> int:

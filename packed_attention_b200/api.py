@@ -23,10 +23,14 @@ def _stream_handle(stream=None):
 
 
 class PackedPlan:
-    """Host plan from ``mf_pack_plan`` plus its device copies."""
+    """Host plan from ``mf_pack_plan`` plus its device copies.
+
+    On a CUDA device the work list is balanced over the device's SMs by
+    ``mf_schedule_work`` (``ctas``: None for the SM count, 0 to keep the
+    plan's cost-ordered list as is)."""
 
     def __init__(self, samples, heads: int, head_dim: int, token_budget: int = 0,
-                 device: torch.device | str = "cuda"):
+                 device: torch.device | str = "cuda", ctas: int | None = None):
         host = _native.pack_plan(samples, heads, head_dim, token_budget)
         self.host = host
         self.samples = [tuple(s) + (1,) * (4 - len(s)) for s in samples]
@@ -34,11 +38,17 @@ class PackedPlan:
         self.total_tokens = host["total_tokens"]
         self.heads = heads
         self.head_dim = head_dim
-        self.n_work = int(host["work"].shape[0])
         self.device = torch.device(device)
+        work = host["work"]
+        if ctas is None and self.device.type == "cuda":
+            ctas = torch.cuda.get_device_properties(self.device).multi_processor_count
+        if ctas:
+            work = _native.schedule_work(work, ctas)
+        self.ctas = int(ctas or 0)
+        self.n_work = int(work.shape[0])
         self.cu_seqlens = torch.from_numpy(host["cu_seqlens"]).to(self.device)
         self.segs = torch.from_numpy(host["segs"]).to(self.device)
-        self.work = torch.from_numpy(host["work"]).to(self.device)
+        self.work = torch.from_numpy(work).to(self.device)
 
     @property
     def seg_lens(self):

@@ -211,7 +211,8 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BwdCtl& ctl, ui
   const int stride = static_cast<int>(gridDim.x);
   int pc = 0, gx = 0, gy = 0;
   bool ok = true;
-  for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+  for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+       idx = next_item(p.work, p.n_work, idx + stride, stride)) {
     const ItemInfo it = load_item(p.segs, p.work, idx);
     const int passes = it.b_valid ? 2 : 1;
     for (int t = 0; t < passes && ok; ++t) {
@@ -262,7 +263,9 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BwdCtl& ctl, ui
 // Passes and steps this CTA will run (for releasing only refilled slots).
 __device__ __forceinline__ void bwd_counts(const BwdParams& p, int& passes, int& steps) {
   passes = steps = 0;
-  for (int idx = blockIdx.x; idx < p.n_work; idx += static_cast<int>(gridDim.x)) {
+  const int stride = static_cast<int>(gridDim.x);
+  for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work;
+       idx = next_item(p.work, p.n_work, idx + stride, stride)) {
     const ItemInfo it = load_item(p.segs, p.work, idx);
     const int np = it.b_valid ? 2 : 1;
     passes += np;
@@ -322,7 +325,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int pc = 0, g = 0;
       uint32_t nph = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+      for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+       idx = next_item(p.work, p.n_work, idx + stride, stride)) {
         const ItemInfo it = load_item(p.segs, p.work, idx);
         const int passes = it.b_valid ? 2 : 1;
         for (int t = 0; t < passes && ok; ++t) {
@@ -387,7 +391,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t ns = 0, nd = 0;
     int pc = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+    for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+       idx = next_item(p.work, p.n_work, idx + stride, stride)) {
       const ItemInfo it = load_item(p.segs, p.work, idx);
       const int passes = it.b_valid ? 2 : 1;
       const int seg_end = it.seg_start + it.seg_len;
@@ -576,7 +581,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int pc = 0, g = 0;
       uint32_t nph = 0, nsf = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+      for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+       idx = next_item(p.work, p.n_work, idx + stride, stride)) {
         const ItemInfo it = load_item(p.segs, p.work, idx);
         const int passes = it.b_valid ? 2 : 1;
         for (int t = 0; t < passes && ok; ++t) {
@@ -643,7 +649,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t ns = 0, nd = 0;
     int pc = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+    for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+       idx = next_item(p.work, p.n_work, idx + stride, stride)) {
       const ItemInfo it = load_item(p.segs, p.work, idx);
       const int passes = it.b_valid ? 2 : 1;
       const int seg_end = it.seg_start + it.seg_len;

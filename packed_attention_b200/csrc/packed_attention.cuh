@@ -147,6 +147,14 @@ __device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int idx) {
   return load_item(p.segs, p.work, idx);
 }
 
+// The first work-list position >= idx in this CTA's stride that holds an
+// item: a scheduled list (mf_schedule_work) pads CTAs that have fewer items
+// with entries of q_tile < 0, which every role skips.
+__device__ __forceinline__ int next_item(const mf_work_item* work, int n_work, int idx, int stride) {
+  while (idx < n_work && work[idx].q_tile < 0) idx += stride;
+  return idx;
+}
+
 struct SharedCtl {
   uint64_t q_full;
   uint64_t q_empty;
@@ -313,7 +321,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int g = 0;  // tile loads issued into the ring so far
       int k = 0;  // items started
       bool ok = true;
-      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride, ++k) {
+      for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+           idx = next_item(p.work, p.n_work, idx + stride, stride), ++k) {
         const ItemInfo it = load_item(p, idx);
         if (k > 0 && !wait_bar(&ctl.q_empty, (k - 1) & 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(&ctl.q_full, 2 * kTile);
@@ -355,14 +364,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // Loads this CTA will consume: a stage is released only if it will be
       // refilled, so that no arrival is left pending when the CTA exits.
       int total_loads = 0;
-      for (int idx = blockIdx.x; idx < p.n_work; idx += stride) total_loads += 2 * load_item(p, idx).n_kv;
+      for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work;
+           idx = next_item(p.work, p.n_work, idx + stride, stride))
+        total_loads += 2 * load_item(p, idx).n_kv;
       int g = 0;        // tile loads consumed so far
       int k = 0;        // items done
       uint32_t np[2] = {0, 0};  // P phases consumed per sub-tile
       bool ok = true;
-      for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride, ++k) {
+      int nidx;
+      for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+           idx = nidx, ++k) {
         const ItemInfo it = load_item(p, idx);
-        const bool has_next = idx + stride < p.n_work;
+        nidx = next_item(p.work, p.n_work, idx + stride, stride);
+        const bool has_next = nidx < p.n_work;
         const int n = it.n_kv;
         const int nt = it.b_valid ? 2 : 1;
         if (!wait_bar(&ctl.q_full, k & 1, abort_flag)) { ok = false; break; }
@@ -438,7 +452,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t ns = 0;  // S phases consumed
     uint32_t no = 0;  // O phases consumed
     bool ok = true;
-    for (int idx = blockIdx.x; idx < p.n_work && ok; idx += stride) {
+    for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+         idx = next_item(p.work, p.n_work, idx + stride, stride)) {
       const ItemInfo it = load_item(p, idx);
       if (t == 1 && !it.b_valid) continue;
       // Rows past the sample end (another sample's tokens, or zeros) are

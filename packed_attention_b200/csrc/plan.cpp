@@ -14,11 +14,14 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <functional>
+#include <queue>
+#include <utility>
 #include <vector>
 
 #include "../../include/mf_attn.h"
 
-extern "C" int32_t mf_abi_version(void) { return 2; }
+extern "C" int32_t mf_abi_version(void) { return 3; }
 
 extern "C" const char* mf_status_string(mf_status status) {
   switch (status) {
@@ -94,5 +97,48 @@ extern "C" mf_status mf_pack_plan(int32_t n_samples, const int32_t* n_text,
       return cost(a) > cost(b);
     });
   }
+  return MF_OK;
+}
+
+extern "C" mf_status mf_schedule_work(const mf_work_item* work, int32_t n_work, int32_t n_ctas,
+                                      mf_work_item* sched, int32_t* n_sched) {
+  if (!work || !n_sched || n_work < 1 || n_ctas < 1) return MF_ERR_INVALID_ARG;
+  const int32_t ctas = std::min(n_ctas, n_work);
+  std::vector<int64_t> cost(static_cast<size_t>(n_work));
+  for (int32_t i = 0; i < n_work; ++i) {
+    const mf_work_item& it = work[i];
+    if (it.q_tile < 0 || it.kv_len < 1) return MF_ERR_INVALID_ARG;
+    const int64_t rows = std::min<int64_t>(MF_TILE_M, int64_t{it.kv_len} - int64_t{it.q_tile} * MF_TILE_M);
+    if (rows < 1) return MF_ERR_INVALID_ARG;
+    const int64_t steps = (int64_t{it.kv_len} + MF_TILE_N - 1) / MF_TILE_N;
+    cost[i] = steps * (rows > MF_TILE_M / 2 ? 20 : 19);
+  }
+  std::vector<int32_t> order(static_cast<size_t>(n_work));
+  for (int32_t i = 0; i < n_work; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return cost[a] > cost[b]; });
+  // least-loaded CTA first, lowest index on ties
+  using Slot = std::pair<int64_t, int32_t>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int32_t c = 0; c < ctas; ++c) heap.push({0, c});
+  std::vector<std::vector<int32_t>> lists(static_cast<size_t>(ctas));
+  size_t rounds = 0;
+  for (const int32_t i : order) {
+    const Slot s = heap.top();
+    heap.pop();
+    lists[s.second].push_back(i);
+    rounds = std::max(rounds, lists[s.second].size());
+    heap.push({s.first + cost[i], s.second});
+  }
+  const int64_t total = static_cast<int64_t>(rounds) * ctas;
+  if (total > INT32_MAX) return MF_ERR_INVALID_ARG;
+  if (!sched) {
+    *n_sched = static_cast<int32_t>(total);
+    return MF_OK;
+  }
+  if (*n_sched < total) return MF_ERR_INVALID_ARG;
+  for (size_t r = 0; r < rounds; ++r)
+    for (int32_t c = 0; c < ctas; ++c)
+      sched[r * ctas + c] = r < lists[c].size() ? work[lists[c][r]] : mf_work_item{0, 0, -1, 0};
+  *n_sched = static_cast<int32_t>(total);
   return MF_OK;
 }

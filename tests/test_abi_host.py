@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    assert lib.mf_abi_version() == 2
+    assert lib.mf_abi_version() == 3
     for code, name in _native.STATUS.items():
         assert lib.mf_status_string(code).decode() == name
 
@@ -226,3 +226,74 @@ def test_diagnostic_entry_points_reject_bad_arguments(lib):
     assert lib.mf_selftest_timeout(2_000_000_000, None) == -1
     assert lib.mf_selftest_exp2(None, None, 4, None) == -1
     assert lib.mf_selftest_exp2(ctypes.c_void_p(16), ctypes.c_void_p(32), -1, None) == -1
+
+
+# ------------------------------------------------------- mf_schedule_work ---
+
+def _lpt_by_hand(work, ctas):
+    """Longest processing time first, written out: cost = key steps x (20 with
+    two query sub-tiles, 19 with one), stable in the input order; each item to
+    the least-loaded CTA, lowest index on ties."""
+    def cost(item):
+        s, h, t, L = item
+        rows = min(pa.MF_TILE_M, L - t * pa.MF_TILE_M)
+        return -(-L // pa.MF_TILE_N) * (20 if rows > pa.MF_TILE_M // 2 else 19)
+    order = sorted(range(len(work)), key=lambda i: -cost(work[i]))
+    load = [0] * ctas
+    lists = [[] for _ in range(ctas)]
+    for i in order:
+        c = min(range(ctas), key=lambda k: (load[k], k))
+        lists[c].append(tuple(work[i]))
+        load[c] += cost(work[i])
+    return lists, load
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 4])
+@pytest.mark.parametrize("ctas", [1, 3, 148])
+def test_schedule_is_lpt_laid_out_for_the_stride(lib, cfg, ctas):
+    w = WORKLOADS[cfg]
+    work = pa.pack_plan(w.samples, w.heads, w.head_dim, w.token_budget)["work"]
+    sched = _native.schedule_work(work, ctas)
+    g = min(ctas, len(work))
+    assert len(sched) % g == 0
+    # every item exactly once; the rest is padding {0, 0, -1, 0}
+    real = sched[sched[:, 2] >= 0]
+    assert sorted(map(tuple, real.tolist())) == sorted(map(tuple, work.tolist()))
+    pad = sched[sched[:, 2] < 0]
+    assert (pad == np.array([0, 0, -1, 0])).all()
+    # CTA c's items sit at c, c + g, ...: its LPT list, then padding only
+    lists, load = _lpt_by_hand(work.tolist(), g)
+    for c in range(g):
+        col = [tuple(x) for x in sched[c::g].tolist()]
+        n = len(lists[c])
+        assert col[:n] == lists[c]
+        assert all(x[2] < 0 for x in col[n:])
+    # never worse than the plain round-robin of the cost-ordered list
+    rr = [0] * g
+    def cost(item):
+        s, h, t, L = item
+        rows = min(pa.MF_TILE_M, L - t * pa.MF_TILE_M)
+        return -(-L // pa.MF_TILE_N) * (20 if rows > pa.MF_TILE_M // 2 else 19)
+    for i, item in enumerate(work.tolist()):
+        rr[i % g] += cost(item)
+    assert max(load) <= max(rr)
+
+
+def test_schedule_arguments(lib):
+    work = pa.pack_plan([(3, 4, 5)], 2, 128)["work"]
+    wp = work.ctypes.data_as(ctypes.c_void_p)
+    n = ctypes.c_int32(0)
+    assert lib.mf_schedule_work(None, len(work), 4, None, ctypes.byref(n)) == -1
+    assert lib.mf_schedule_work(wp, 0, 4, None, ctypes.byref(n)) == -1
+    assert lib.mf_schedule_work(wp, len(work), 0, None, ctypes.byref(n)) == -1
+    assert lib.mf_schedule_work(wp, len(work), 4, None, None) == -1
+    assert lib.mf_schedule_work(wp, len(work), 4, None, ctypes.byref(n)) == 0
+    assert n.value == 2  # 2 items, CTAs capped at 2: one round
+    out = np.zeros((1, 4), dtype=np.int32)
+    small = ctypes.c_int32(1)
+    assert lib.mf_schedule_work(wp, len(work), 4, out.ctypes.data_as(ctypes.c_void_p),
+                                ctypes.byref(small)) == -1
+    bad = work.copy()
+    bad[1, 2] = -1  # a padding entry is not an input item
+    assert lib.mf_schedule_work(bad.ctypes.data_as(ctypes.c_void_p), len(bad), 4, None,
+                                ctypes.byref(n)) == -1
