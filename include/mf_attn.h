@@ -178,7 +178,8 @@ mf_status mf_qk_prologue(const void* q, const void* k, const float* g_q_text,
  * measurement: block-diagonal softmax attention of q_hat, k_hat (read from
  * the workspace that mf_qk_prologue filled) and v, on tensor cores.
  *   v              bf16 [total_tokens, heads, head_dim], contiguous, 16-B aligned
- *   work_dev       mf_work_item [n_work], device, from mf_pack_plan
+ *   work_dev       mf_work_item [n_work], device, from mf_pack_plan, or laid
+ *                  out by mf_schedule_work (entries with q_tile < 0 are skipped)
  *   softmax_scale  <= 0 selects 1/sqrt(head_dim)
  *   out            bf16 [total_tokens, heads, head_dim], 16-B aligned, must not
  *                  overlap q, k, v or the workspace
