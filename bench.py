@@ -35,7 +35,7 @@ KERNEL_SOURCE = os.path.join(ROOT, "packed_attention_b200", "csrc", "packed_atte
 # the full workload (profiles/traffic_packed_attention_kernel_*.md), keyed by
 # the kernel source it was taken on: any other source reports null.
 MEASURED_TRAFFIC = {
-    ("ac77df845750b2a0", "hires_2048sq_4to1"): 399_218_688 + 110_845_184,
+    ("9a964a1d1e73aba6", "hires_2048sq_4to1"): 399_032_320 + 109_391_872,
 }
 
 
