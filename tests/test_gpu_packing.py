@@ -75,3 +75,34 @@ def test_each_sample_alone_is_bitwise_equal(cuda_device, trial):
         _, _, oi = run_gpu(wi, gather_inputs(inp, tok), cuda_device)
         assert np.array_equal(packed[tok], bits(oi)), i
         start += L
+
+
+def test_schedule_does_not_change_results(cuda_device):
+    """The work list's schedule (mf_schedule_work over any number of CTAs,
+    with its padding entries, or none) only moves whole items between CTAs:
+    forward, log-normaliser and backward are bit-identical."""
+    w = Workload("sched", ((77, 12, 20, 1), (0, 9, 15, 1), (5, 1, 1, 1), (200, 8, 8, 2),
+                           (31, 1, 1, 1)), heads=3, head_dim=128, seed=18)
+    inp = make_inputs(w)
+    t = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).to(cuda_device)
+         for n in ("q", "k", "v")}
+    t.update({n: torch.from_numpy(inp[n]).to(cuda_device) for n in pa.GAMMA_NAMES})
+    dout = torch.from_numpy(
+        np.random.default_rng(3).standard_normal(t["q"].shape).astype(np.float32)).to(
+        cuda_device).to(torch.bfloat16)
+    results = []
+    for ctas in (0, None, 1, 5, 37, 1000):
+        plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, device=cuda_device, ctas=ctas)
+        if ctas == 5:
+            assert (plan.work[:, 2] < 0).any()  # the padded layout is exercised
+        out, lse = pa.joint_attention_fwd_lse(t["q"], t["k"], t["v"], t, plan, eps=w.eps)
+        g = pa.joint_attention_bwd(t["q"], t["k"], t["v"], t, plan, out, lse, dout, eps=w.eps)
+        assert pa.device_error() == 0
+        results.append((bits(out), lse.cpu().numpy(), bits(g["dq"]), bits(g["dk"]),
+                        bits(g["dv"]), [g[n].cpu().numpy() for n in pa.GAMMA_NAMES]))
+    ref = results[0]
+    for r in results[1:]:
+        for a, b in zip(ref[:5], r[:5]):
+            assert np.array_equal(a, b)
+        for a, b in zip(ref[5], r[5]):
+            assert np.array_equal(a, b)

@@ -133,6 +133,22 @@ def test_small_pack_full_compare(cuda_device, name, w):
     assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
 
 
+def test_long_sample_sampled_rows(cuda_device):
+    """One sample of 131,072 tokens: 512 work items of 1,024 key steps each,
+    on sampled rows (the first, the last, 96 random tokens, both heads)."""
+    w = Workload("long_131k", ((0, 256, 512, 1),), heads=2, head_dim=128, seed=19)
+    inp = make_inputs(w)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    rng = np.random.default_rng(11)
+    toks = np.unique(np.concatenate([[0, 1, w.total_tokens - 1],
+                                     rng.choice(w.total_tokens, 96, replace=False)]))
+    rows = (toks[:, None] * w.heads + np.arange(w.heads)[None, :]).reshape(-1)
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
+    got = bf16_to_f64(out).reshape(-1, w.head_dim)[rows]
+    max_abs, rel_rms = errors(got, ref)
+    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
+
+
 @pytest.mark.parametrize("trial", range(4))
 def test_random_packs_full_compare(cuda_device, trial):
     rng = np.random.default_rng(500 + trial)
