@@ -6,9 +6,10 @@ in ``include/mf_attn.h``); this package marshals torch tensors into it.
 Importing the package does not load the library; the first call does, and
 raises if the library has not been built.
 """
-from ._native import MfError, MF_TILE_M, MF_TILE_N, pack_plan, workspace_bytes  # noqa: F401
+from ._native import (MfError, MF_TILE_M, MF_TILE_N, pack_plan, schedule_work,  # noqa: F401
+                      workspace_bytes)
 
-__all__ = ["MfError", "MF_TILE_M", "MF_TILE_N", "pack_plan", "workspace_bytes",
+__all__ = ["MfError", "MF_TILE_M", "MF_TILE_N", "pack_plan", "schedule_work", "workspace_bytes",
            "PackedPlan", "joint_attention", "joint_attention_host", "qk_prologue",
            "packed_attention", "workspace_views", "device_error", "joint_attention_fwd_lse",
            "joint_attention_bwd", "joint_attention_autograd", "bwd_workspace_bytes",
