@@ -33,17 +33,27 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCE = os.path.join(ROOT, "packed_attention_b200", "csrc", "packed_attention.cuh")
 # DRAM bytes (read + write) of one attention launch, from one ncu capture of
 # the full workload (profiles/traffic_packed_attention_kernel_*.md), keyed by
-# the kernel source it was taken on: any other source reports null.
+# the kernel code it was taken on (the sha256 of the source with comments and
+# blank lines removed, so that a comment edit keeps the figure): any other
+# code reports null.
 MEASURED_TRAFFIC = {
-    ("9a964a1d1e73aba6", "hires_2048sq_4to1"): 399_032_320 + 109_391_872,
+    ("b9c3dbf84302795b", "hires_2048sq_4to1"): 399_032_320 + 109_391_872,
 }
 
 
-def kernel_traffic(workload_name):
+def kernel_code_sha(path=KERNEL_SOURCE):
     import hashlib
-    with open(KERNEL_SOURCE, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    return MEASURED_TRAFFIC.get((sha, workload_name))
+    import re
+    with open(path) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in src.splitlines()]
+    code = "\n".join(ln for ln in lines if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
+def kernel_traffic(workload_name):
+    return MEASURED_TRAFFIC.get((kernel_code_sha(), workload_name))
 
 
 def parse_args():

@@ -6,8 +6,10 @@
 //  cumulative offsets. The pages run it with FlashAttention's var-len
 //  kernels; this kernel is its own design for sm_100a.]
 //
-// Persistent: one CTA per SM walks the longest-first work list with a
-// stride of gridDim.x. A work item is 256 query rows of one head of one
+// Persistent: one CTA per SM walks the work list with a stride of
+// gridDim.x (a list laid out by mf_schedule_work gives each CTA its share of
+// a longest-processing-time-first balance; its padding entries are skipped).
+// A work item is 256 query rows of one head of one
 // sample, split into two 128-row sub-tiles a and b that share every K/V tile
 // (b is skipped when it starts past the sample end). Keys are visited in
 // steps of 128.
@@ -19,7 +21,9 @@
 //                    when the running max of a row inside the sample grew by
 //                    more than 2^8 (a stale max keeps p <= 256: exact enough
 //                    in bf16, safe in fp32). At the end of an item: O / l ->
-//                    bf16 rows, skipping rows past the sample end.
+//                    bf16 rows through 4 KB of shared memory per warp, so
+//                    that the stores write whole 128-byte row segments,
+//                    skipping rows past the sample end.
 //   warp 8 (1 lane)  TMA producer: both Q sub-tiles per item, then K_j, V_j
 //                    into a ring of shared-memory stages (128-byte swizzled
 //                    boxes of 128 rows x 64 dims).
