@@ -190,3 +190,35 @@ def test_autograd_function_matches_the_direct_call(cuda_device):
     grads = torch.autograd.grad(o, leaves, dout)
     for x, key in zip(grads, ("dq", "dk", "dv") + NAMES):
         assert torch.equal(x, g[key]), key
+
+
+@pytest.mark.parametrize("trial", range(12))
+def test_fwd_bwd_sweep_small_packs(cuda_device, trial):
+    """Small random packs over the whole space: 1-6 samples, 0-64 text tokens,
+    grids up to 12 per side, 1-3 frames, d 64 or 128, 1-3 heads, frame dims
+    0/4/8/16, and the work list scheduled for the SM count, for 3 CTAs or not
+    at all. Forward output, log-normaliser and every gradient against the
+    oracle."""
+    rng = np.random.default_rng(4100 + trial)
+    samples = random_pack(rng, int(rng.integers(1, 7)), 64, 12, 3)
+    d = (64, 128)[trial % 2]
+    w = Workload(f"sweep_{trial}", samples, heads=int(rng.integers(1, 4)), head_dim=d,
+                 seed=4200 + trial, rope_frame_dims=(0, 4, 8, 16)[trial % 4])
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    ctas = (None, 0, 3)[trial % 3]
+    plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, device=cuda_device, ctas=ctas)
+    t = to_dev(inp, cuda_device)
+    out, lse = pa.joint_attention_fwd_lse(t["q"], t["k"], t["v"], t, plan, eps=w.eps,
+                                          frame_dims=w.rope_frame_dims)
+    dout = torch.from_numpy(dob.view(np.int16)).view(torch.bfloat16).to(cuda_device)
+    g = pa.joint_attention_bwd(t["q"], t["k"], t["v"], t, plan, out, lse, dout, eps=w.eps,
+                               frame_dims=w.rope_frame_dims)
+    assert pa.device_error() == 0
+    ref = oracle_grads(w, inp, dob)
+    o = bf16_to_f64(out)
+    err = o - ref["out"]
+    rms = float(np.sqrt(np.mean(ref["out"] ** 2)))
+    assert float(np.max(np.abs(err))) <= 2e-2 and float(np.sqrt(np.mean(err ** 2))) / rms <= 5e-3
+    assert float(np.max(np.abs(lse.double().cpu().numpy() - ref["lse"].T))) < 1e-2
+    check_grads(w.name, g, ref)
