@@ -53,7 +53,7 @@ typedef enum {
   MF_ERR_INVALID_ARG = -1, /* NULL pointer, negative or inconsistent size      */
   MF_ERR_UNSUPPORTED = -2, /* head_dim not in {64, 128}                         */
   MF_ERR_ALIGNMENT = -3,   /* a device pointer is not 16-byte aligned           */
-  MF_ERR_WORKSPACE = -4,   /* workspace_bytes < mf_workspace_bytes(...)         */
+  MF_ERR_WORKSPACE = -4,   /* workspace smaller than the *_workspace_bytes query  */
   MF_ERR_BUDGET = -5,      /* total tokens exceed the pack's token budget       */
   MF_ERR_CUDA = -6,        /* a CUDA runtime or driver call failed              */
   MF_ERR_TIMEOUT = -7      /* a kernel pipeline wait ran out of time            */
@@ -147,24 +147,24 @@ mf_status mf_schedule_work(const mf_work_item* work, int32_t n_work, int32_t n_c
                            mf_work_item* sched, int32_t* n_sched);
 
 /*
- * Bytes of device workspace mf_joint_attn_fwd needs: the normalised, rotated
- * q_hat and k_hat ([T, H, d] bf16 each) plus a small control block.
+ * mf_joint_attn_workspace_bytes -- bytes of device workspace mf_joint_attn_fwd
+ * (and its stages) needs: the normalised, rotated q_hat and k_hat
+ * ([T, H, d] bf16 each, each padded to a multiple of 256 bytes).
  * Returns 0 for invalid sizes.
  */
-size_t mf_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim);
+size_t mf_joint_attn_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim);
 
 /*
  * mf_qk_prologue -- stage 1 of mf_joint_attn_fwd, exposed for measurement.
  * For every token and head, RMSNorm q and k with the gamma of the token's
  * modality and rotate image tokens by their grid position (see the readings
- * above); writes q_hat and k_hat (bf16, [T, H, d]) into the workspace and
- * resets the work-list counter the attention stage pops from.
+ * above); writes q_hat and k_hat (bf16, [T, H, d]) into the workspace.
  *   q, k           bf16 [total_tokens, heads, head_dim], contiguous, 16-B aligned
  *   g_q_text ...   fp32 [head_dim] each, device
  *   cu_seqlens_dev int32 [n_samples + 1], device, from mf_pack_plan
  *   segs_dev       mf_segment [n_samples], device, from mf_pack_plan
  *   eps            added to the mean square (e.g. 1e-6), must be >= 0
- *   workspace      device, >= mf_workspace_bytes(...), 256-B aligned
+ *   workspace      device, >= mf_joint_attn_workspace_bytes(...), 256-B aligned
  */
 mf_status mf_qk_prologue(const void* q, const void* k, const float* g_q_text,
                          const float* g_q_img, const float* g_k_text, const float* g_k_img,
@@ -346,13 +346,17 @@ mf_status mf_attn_block_fwd(const void* h, const float* shift, const float* scal
  * calls no allocating routine. Arguments are those of mf_joint_attn_fwd
  * without workspace / workspace_bytes; inputs and outputs are still the
  * caller's.
- *   - Packs whose scratch need, mf_workspace_bytes(total_tokens, heads,
- *     head_dim), exceeds MF_STATIC_SCRATCH_BYTES are rejected with
+ *   - Packs whose scratch need, mf_joint_attn_workspace_bytes(total_tokens,
+ *     heads, head_dim), exceeds MF_STATIC_SCRATCH_BYTES are rejected with
  *     MF_ERR_WORKSPACE before anything is launched (64 MiB holds q_hat and
  *     k_hat for up to ~131,000 (token, head) rows at head_dim 128).
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture begins.
+ *     before any stream capture begins. The address is kept once a lookup
+ *     has succeeded (a failed lookup returns MF_ERR_CUDA and is retried by
+ *     the next call). cudaDeviceReset unloads the library's device code and
+ *     with it the array: after a reset of a device, do not call this entry
+ *     point on that device again in the same process.
  *   - All calls share the one array, and it keeps whatever the last call
  *     left in it (every call rewrites the parts it reads). Calls whose
  *     kernels overlap on the GPU -- on two streams, or from two threads --
@@ -368,12 +372,12 @@ mf_status mf_joint_attn_fwd_static_scratch(
     void* out, void* stream);
 
 /*
- * mf_selftest_exp2 -- diagnostic: y[i] = 2^x[i] computed by the attention
- * softmax's FMA-pipe exponential (the share of exponentials it keeps off the
- * MUFU unit), so its accuracy can be checked on its own. x, y: device fp32
- * arrays of n elements (n >= 0; n odd is fine). Inputs below -125 give
- * 2^-125-scale values (zero to bf16), -inf included. Asynchronous on
- * `stream`; MF_ERR_INVALID_ARG for NULL pointers or n < 0.
+ * mf_selftest_exp2 -- diagnostic: y[i] = 2^x[i] computed by the same
+ * instruction the attention softmax uses for its exponentials (the MUFU
+ * unit's approximate exp2, denormal results flushed to zero), so that its
+ * accuracy can be checked on its own. x, y: device fp32 arrays of n elements
+ * (n >= 0). Asynchronous on `stream`; MF_ERR_INVALID_ARG for NULL pointers
+ * or n < 0.
  */
 mf_status mf_selftest_exp2(const float* x, float* y, int32_t n, void* stream);
 

@@ -55,7 +55,7 @@ SIGNATURES = {
     "mf_status_string": (ctypes.c_char_p, [I32]),
     "mf_pack_plan": (I32, [I32, P, P, P, P, I32, I32, I64, P, P, P, P, P]),
     "mf_schedule_work": (I32, [P, I32, I32, P, P]),
-    "mf_workspace_bytes": (SZ, [I32, I32, I32]),
+    "mf_joint_attn_workspace_bytes": (SZ, [I32, I32, I32]),
     "mf_qk_prologue": (I32, [P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, P, SZ, P]),
     "mf_qk_prologue_3d": (I32, [P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, I32, P, SZ, P]),
     "mf_packed_attention": (I32, [P, P, I32, P, I32, I32, I32, I32, F32, P, P, SZ, P]),
@@ -144,4 +144,4 @@ def schedule_work(work, n_ctas: int):
 
 
 def workspace_bytes(total_tokens: int, heads: int, head_dim: int) -> int:
-    return int(lib().mf_workspace_bytes(total_tokens, heads, head_dim))
+    return int(lib().mf_joint_attn_workspace_bytes(total_tokens, heads, head_dim))

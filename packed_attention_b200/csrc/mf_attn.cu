@@ -22,7 +22,6 @@
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr size_t kCtlBytes = 256;
 constexpr int kMaxDevices = 64;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -30,7 +29,6 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct WorkspaceLayout {
   size_t q_hat;
   size_t k_hat;
-  size_t ctl;
   size_t total;
 };
 
@@ -39,8 +37,7 @@ bool layout(int32_t total_tokens, int32_t heads, int32_t head_dim, WorkspaceLayo
   const size_t tensor = round_up(static_cast<size_t>(total_tokens) * heads * head_dim * 2, kAlign);
   w->q_hat = 0;
   w->k_hat = tensor;
-  w->ctl = 2 * tensor;
-  w->total = 2 * tensor + kCtlBytes;
+  w->total = 2 * tensor;
   return true;
 }
 
@@ -148,7 +145,7 @@ bool prepare_bwd_kernels() {
   return ok[dev];
 }
 
-// Backward workspace: the forward's (q_hat, k_hat, control block), then
+// Backward workspace: the forward's (q_hat, k_hat), then
 // D [H, T] fp32, dq_hat and dk_hat [T, H, d] fp32 and the per-block partial
 // gamma gradients [blocks, 4, d] fp32.
 struct BwdLayout {
@@ -172,7 +169,7 @@ bool bwd_layout(int32_t total_tokens, int32_t heads, int32_t head_dim, BwdLayout
 
 }  // namespace
 
-extern "C" size_t mf_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim) {
+extern "C" size_t mf_joint_attn_workspace_bytes(int32_t total_tokens, int32_t heads, int32_t head_dim) {
   WorkspaceLayout w;
   return layout(total_tokens, heads, head_dim, &w) ? w.total : 0;
 }
@@ -205,17 +202,16 @@ extern "C" mf_status mf_qk_prologue_3d(const void* q, const void* k, const float
   const int vec_per_row = head_dim / 8;
   const int tok_per_block = mf::kPrologueThreads / vec_per_row;
   const unsigned grid = static_cast<unsigned>((total_tokens + tok_per_block - 1) / tok_per_block);
-  auto* counter = reinterpret_cast<int32_t*>(ws + w.ctl);
   if (head_dim == 128) {
     mf::qk_prologue_kernel<128><<<grid, mf::kPrologueThreads, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
         g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims,
-        reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat), counter);
+        reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat));
   } else {
     mf::qk_prologue_kernel<64><<<grid, mf::kPrologueThreads, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
         g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims,
-        reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat), counter);
+        reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat));
   }
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
 }
@@ -347,14 +343,10 @@ extern "C" mf_status mf_joint_attn_fwd(const void* q, const void* k, const void*
 
 namespace {
 
+// y = 2^x through the same instruction the softmax uses for its exponentials.
 __global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.0f;
-  float y0, y1;
-  mf::exp2_fma_x2(x0, x1, y0, y1);
-  y[i] = y0;
-  if (i + 1 < n) y[i + 1] = y1;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = mf::ex2_approx(x[i]);
 }
 
 }  // namespace
@@ -362,8 +354,7 @@ __global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restr
 extern "C" mf_status mf_selftest_exp2(const float* x, float* y, int32_t n, void* stream) {
   if (!x || !y || n < 0) return MF_ERR_INVALID_ARG;
   if (n == 0) return MF_OK;
-  const int pairs = (n + 1) / 2;
-  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;
 }
 

@@ -91,8 +91,6 @@ constexpr int kBoxBytes = 128 * 128;   // 128 rows x 64 bf16 = one 128-byte swiz
 constexpr int kMaxStages = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// One column pair in kPolyEvery takes its exponentials on the FMA pipe (0: none).
-constexpr int kPolyEvery = 0;
 
 static_assert(MF_TILE_M == 2 * kSubM, "a work item is two query sub-tiles");
 
@@ -203,31 +201,6 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
                                               volatile int32_t* abort_flag) {
   const bool ok = wait_bar(bar, parity, abort_flag);
   return __all_sync(0xffffffffu, ok);
-}
-
-// 2^x for two lanes on the FMA pipe, to take a share of the exponentials off
-// the MUFU unit (whose 16 results per clock per SM equal the tensor core's
-// score rate). Cody-Waite reduction x = n + f, n = rint(x), f in [-1/2, 1/2]
-// (rint by adding 1.5 * 2^23), 2^f by a cubic with minimax relative error
-// 7.5e-5 (coefficients from fit_exp2_poly.py), and 2^n added to the exponent
-// field with one integer multiply-add. x is clamped at -125 so that n + the
-// exponent of 2^f stays a normal exponent (2^-125 ~ 2.4e-38 is zero to bf16).
-__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
-  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
-  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t x = f32x2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t xr = add_f32x2(x, f32x2(kRound, kRound));        // n in the low mantissa bits
-  const uint64_t n = add_f32x2(xr, f32x2(-kRound, -kRound));      // rint(x)
-  const uint64_t f = fma_f32x2(n, f32x2(-1.0f, -1.0f), x);        // x - n, exact
-  uint64_t q = fma_f32x2(f32x2(kC3, kC3), f, f32x2(kC2, kC2));
-  q = fma_f32x2(q, f, f32x2(kC1, kC1));
-  q = fma_f32x2(q, f, f32x2(kC0, kC0));
-  float q0, q1, r0, r1;
-  f32x2_split(q, q0, q1);
-  f32x2_split(xr, r0, r1);
-  y0 = __uint_as_float(imad(__float_as_uint(r0), 1u << 23, __float_as_uint(q0)));
-  y1 = __uint_as_float(imad(__float_as_uint(r1), 1u << 23, __float_as_uint(q1)));
 }
 
 // Shared-memory descriptors are built once; a descriptor for base + off is
@@ -522,14 +495,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < 32; ++c) {
             const int e = 64 * h + 2 * c;
             const uint64_t x = fma_f32x2(f32x2(s[e], s[e + 1]), sl2x2, neg_m);
-            float x0, x1, p0, p1;
+            float x0, x1;
             f32x2_split(x, x0, x1);
-            if (kPolyEvery > 0 && c % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
-              exp2_fma_x2(x0, x1, p0, p1);  // a share of the exponentials on the FMA pipe
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             // Row sum in four scalar chains (packing p0, p1 for a paired add
             // would cost register moves).
             if (c & 1) { la1 += p0; lb1 += p1; } else { la0 += p0; lb0 += p1; }

@@ -21,7 +21,7 @@
 
 #include "../../include/mf_attn.h"
 
-extern "C" int32_t mf_abi_version(void) { return 3; }
+extern "C" int32_t mf_abi_version(void) { return 4; }
 
 extern "C" const char* mf_status_string(mf_status status) {
   switch (status) {

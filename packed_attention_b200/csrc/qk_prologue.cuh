@@ -59,13 +59,10 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
     const float* __restrict__ gq_img, const float* __restrict__ gk_text,
     const float* __restrict__ gk_img, const int32_t* __restrict__ cu_seqlens,
     const mf_segment* __restrict__ segs, int n_samples, int total_tokens, int heads, float eps,
-    int frame_dims, uint4* __restrict__ q_hat, uint4* __restrict__ k_hat,
-    int32_t* __restrict__ work_counter) {
+    int frame_dims, uint4* __restrict__ q_hat, uint4* __restrict__ k_hat) {
   constexpr int kVecPerRow = D / 8;                          // 16-byte vectors per row
   constexpr int kTokPerBlock = kPrologueThreads / kVecPerRow;
   const int spatial = (D - frame_dims) / 2;  // dims per grid axis
-
-  if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
 
   const int vec = threadIdx.x % kVecPerRow;
   const int t_raw = blockIdx.x * kTokPerBlock + threadIdx.x / kVecPerRow;

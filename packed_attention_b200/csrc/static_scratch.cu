@@ -2,15 +2,15 @@
 // allocate device memory (a plugin handed a stream but no allocator, code
 // inside a global-mode stream capture where cudaMalloc is illegal, or a
 // latency-critical loop that cannot pay for cudaMalloc's implicit device
-// synchronisation). The scratch the forward needs (q_hat, k_hat and the
-// control block) comes from a fixed array compiled into the library instead
-// of from the caller. Nothing here allocates: no cudaMalloc, no cudaFree, no
-// allocating library call.
+// synchronisation). The scratch the forward needs (q_hat and k_hat) comes
+// from a fixed array compiled into the library instead of from the caller.
+// Nothing here allocates: no cudaMalloc, no cudaFree, no allocating library
+// call.
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
-#include <mutex>
 
 #include "../../include/mf_attn.h"
 
@@ -24,23 +24,26 @@ constexpr int kMaxDevices = 64;
 // must come from cudaGetSymbolAddress (below), never from taking &g_scratch.
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-struct DeviceScratch {
-  std::once_flag once;
-  void* ptr = nullptr;
-};
-DeviceScratch g_device_scratch[kMaxDevices];
+// Device address of g_scratch per device, cached only once a lookup has
+// succeeded: a failed lookup (for example one attempted while the stream is
+// being captured) leaves the slot empty, and the next call tries again.
+std::atomic<void*> g_scratch_ptr[kMaxDevices];
 
-// Device address of g_scratch on the current device, looked up once per
-// device (with that device current) and cached; NULL if the lookup failed.
+// Address of g_scratch on the current device (looked up with that device
+// current), or NULL if the lookup failed; the failure's error state is
+// cleared so that it does not surface at an unrelated later call.
 void* scratch_on_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  DeviceScratch& d = g_device_scratch[dev];
-  std::call_once(d.once, [&d] {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) == cudaSuccess) d.ptr = p;
-  });
-  return d.ptr;
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  // Two threads may both look it up; they find the same address.
+  g_scratch_ptr[dev].store(p, std::memory_order_release);
+  return p;
 }
 
 }  // namespace
@@ -53,11 +56,13 @@ extern "C" mf_status mf_joint_attn_fwd_static_scratch(
     void* out, void* stream) {
   // Size first: a pack that does not fit is refused before anything runs.
   // (Invalid sizes give 0 here and are reported by mf_joint_attn_fwd.)
-  if (mf_workspace_bytes(total_tokens, heads, head_dim) > kScratchBytes) return MF_ERR_WORKSPACE;
+  if (mf_joint_attn_workspace_bytes(total_tokens, heads, head_dim) > kScratchBytes)
+    return MF_ERR_WORKSPACE;
   void* scratch = scratch_on_current_device();
   if (!scratch) return MF_ERR_CUDA;
-  // The prologue overwrites q_hat, k_hat and resets the control block on
-  // every call, so whatever an earlier call left in the array is never read.
+  // The prologue overwrites q_hat and k_hat on every call before the
+  // attention kernel reads them, so whatever an earlier call left in the
+  // array is never read.
   return mf_joint_attn_fwd(q, k, v, g_q_text, g_q_img, g_k_text, g_k_img, cu_seqlens_dev,
                            segs_dev, n_samples, work_dev, n_work, total_tokens, heads, head_dim,
                            eps, softmax_scale, out, scratch, kScratchBytes, stream);

@@ -40,8 +40,27 @@ def test_every_declared_symbol_is_exported(lib):
     assert sorted(_native.SIGNATURES) == names
 
 
+# The boundary's calls, by name: the operation's own (plan, schedule, workspace
+# query, the two stages and the joint forward), its 3D-rotation, training and
+# sub-layer variants, the allocation-free variant, and the diagnostics.
+DOCUMENTED_ABI = sorted([
+    "mf_abi_version", "mf_status_string",
+    "mf_pack_plan", "mf_schedule_work", "mf_joint_attn_workspace_bytes",
+    "mf_qk_prologue", "mf_packed_attention", "mf_joint_attn_fwd",
+    "mf_qk_prologue_3d", "mf_joint_attn_fwd_3d",
+    "mf_joint_attn_fwd_lse", "mf_bwd_workspace_bytes", "mf_joint_attn_bwd",
+    "mf_block_workspace_bytes", "mf_attn_block_fwd",
+    "mf_joint_attn_fwd_static_scratch",
+    "mf_selftest_exp2", "mf_selftest_timeout", "mf_get_device_error",
+])
+
+
+def test_header_declares_the_documented_calls():
+    assert header_functions() == DOCUMENTED_ABI
+
+
 def test_status_strings(lib):
-    assert lib.mf_abi_version() == 3
+    assert lib.mf_abi_version() == 4
     for code, name in _native.STATUS.items():
         assert lib.mf_status_string(code).decode() == name
 
@@ -126,7 +145,7 @@ def test_plan_two_call_capacity(lib):
 
 
 def test_workspace_size(lib):
-    assert pa.workspace_bytes(152, 2, 64) == 2 * ((152 * 2 * 64 * 2 + 255) // 256 * 256) + 256
+    assert pa.workspace_bytes(152, 2, 64) == 2 * ((152 * 2 * 64 * 2 + 255) // 256 * 256)
     assert pa.workspace_bytes(0, 2, 64) == 0
     assert pa.workspace_bytes(10, 2, 96) == 0
 
@@ -202,7 +221,7 @@ def test_backward_argument_checks(lib):
     need = lib.mf_bwd_workspace_bytes(T, H, d)
     rows = T * H
     r256 = lambda x: (x + 255) // 256 * 256
-    fwd = lib.mf_workspace_bytes(T, H, d)
+    fwd = lib.mf_joint_attn_workspace_bytes(T, H, d)
     blocks = (T + 31) // 32  # 256 threads, 8 per token at d = 64
     assert need == r256(fwd) + r256(rows * 4) + 2 * r256(rows * d * 4) + r256(blocks * 4 * d * 4)
     assert lib.mf_bwd_workspace_bytes(T, H, 96) == 0

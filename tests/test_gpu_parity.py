@@ -3,13 +3,16 @@
 Bar: max-abs error <= 2e-2 and relative RMS error <= 5e-3 over the compared
 elements (bf16 output, fp32 accumulation); the prologue's q_hat / k_hat
 within one bf16 rounding of the oracle. Small packs are compared element by
-element in full; the five full-size packs run in the same launch
-configuration the benchmark times and are compared on sampled rows (every
-segment's first and last rows, tile boundaries, ragged tails and random
-rows).
+element in full. The five full-size packs run in the same launch
+configuration the benchmark times and are compared on every element of the
+output (the oracle's full output is cached on disk per workload) and, as a
+fast smoke, on sampled rows (every segment's first and last rows, tile
+boundaries, ragged tails and random rows).
 """
+import hashlib
 import json
 import os
+import time
 
 import numpy as np
 import pytest
@@ -184,6 +187,79 @@ def test_full_size_config_sampled_rows(cuda_device, cfg):
     assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
 
 
+# ----------------------------------------- full-size packs, every element ---
+
+CACHE_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), ".oracle_cache")
+
+
+def _cache_key(w: Workload) -> str:
+    """Changes whenever the oracle's code, the input generator or the workload
+    (shapes, seed, value recipe) changes."""
+    h = hashlib.sha256(repr(w).encode())
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for rel in ("oracle/oracle.cpp", "packed_attention_b200/synth.py",
+                "packed_attention_b200/workloads.py"):
+        with open(os.path.join(root, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def oracle_full_output(w: Workload, inp):
+    """The oracle's whole ``[T, H, d]`` output for workload ``w`` (fp64
+    arithmetic on all host cores), cached on disk as fp32 under
+    ``tests/.oracle_cache`` so that a rerun on the same machine only reads it
+    back. fp32 storage moves a value by at most 2^-24 relative, five orders of
+    magnitude below the tolerances it is compared at."""
+    path = os.path.join(CACHE_DIR, f"{w.name}-{_cache_key(w)}.npy")
+    if os.path.exists(path):
+        return np.load(path).astype(np.float64), 0.0
+    t0 = time.perf_counter()
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps)
+    sec = time.perf_counter() - t0
+    os.makedirs(CACHE_DIR, exist_ok=True)
+    tmp = path + f".tmp{os.getpid()}.npy"
+    np.save(tmp, ref.astype(np.float32))
+    os.replace(tmp, path)
+    return ref, sec
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_full_size_config_every_element(cuda_device, cfg):
+    """Every element of the full-size pack's output against the oracle: the
+    bar over all T*H*d elements, and the same bar on each head alone (so that
+    an error confined to some heads cannot hide in the average)."""
+    w = WORKLOADS[cfg]
+    inp = make_inputs(w)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    got = out.float().cpu().numpy()
+    del out
+    assert np.all(np.isfinite(got))
+    ref, oracle_s = oracle_full_output(w, inp)
+    sq_diff = sq_ref = 0.0
+    max_abs = 0.0
+    per_head = []
+    for h in range(w.heads):
+        d = got[:, h, :].astype(np.float64) - ref[:, h, :]
+        r = ref[:, h, :]
+        hd, hr, hm = float(np.sum(d * d)), float(np.sum(r * r)), float(np.max(np.abs(d)))
+        per_head.append((hm, float(np.sqrt(hd / hr))))
+        sq_diff += hd
+        sq_ref += hr
+        max_abs = max(max_abs, hm)
+    rel_rms = float(np.sqrt(sq_diff / sq_ref))
+    report = os.environ.get("MF_PARITY_REPORT")
+    if report:
+        with open(report, "a") as f:
+            f.write(json.dumps({"config": cfg, "workload": w.name, "compared": "every element",
+                                "elements": int(got.size), "max_abs": max_abs,
+                                "rel_rms": rel_rms,
+                                "worst_head_rel_rms": max(r for _, r in per_head),
+                                "oracle_seconds": oracle_s}) + "\n")
+    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
+    bad = [(h, m, r) for h, (m, r) in enumerate(per_head) if m > MAX_ABS or r > REL_RMS]
+    assert not bad, bad
+
+
 # --------------------------------------------------------------- hygiene ---
 
 def test_canary_rows_untouched_and_deterministic(cuda_device):
@@ -236,9 +312,12 @@ def test_explicit_softmax_scale(cuda_device):
         assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (scale, max_abs, rel_rms)
 
 
-def test_fma_pipe_exp2_accuracy(cuda_device):
-    """The softmax's polynomial exp2 (Cody-Waite reduction + minimax cubic)
-    against fp64: relative error below 1e-4 wherever the result is normal."""
+def test_softmax_exp2_accuracy(cuda_device):
+    """The exponential the softmax uses (the MUFU unit's approximate exp2)
+    against fp64: relative error below 1e-5 wherever the result is a normal
+    number, i.e. far below the 2^-9 relative rounding of P to bf16, so the
+    approximation costs nothing measurable in the attention output. Results
+    below the normal range flush to zero (the softmax's masked keys use -inf)."""
     import ctypes
     from packed_attention_b200 import _native
     xs = np.concatenate([np.linspace(-125.0, 8.0, 1_000_001), np.arange(-125, 9, dtype=np.float64),
@@ -251,14 +330,12 @@ def test_fma_pipe_exp2_accuracy(cuda_device):
     got = y.cpu().numpy().astype(np.float64)
     ref = np.exp2(x.cpu().numpy().astype(np.float64))
     rel = np.abs(got / ref - 1.0)
-    assert rel.max() < 1e-4, rel.max()
-    # below the clamp, and for -inf, the result is a tiny positive normal number
-    x2 = torch.tensor([-126.0, -200.0, -float("inf"), -3e38], dtype=torch.float32, device=cuda_device)
+    assert rel.max() < 1e-5, rel.max()
+    x2 = torch.tensor([-130.0, -200.0, -float("inf"), -3e38], dtype=torch.float32, device=cuda_device)
     y2 = torch.empty_like(x2)
     assert _native.lib().mf_selftest_exp2(ctypes.c_void_p(x2.data_ptr()), ctypes.c_void_p(y2.data_ptr()),
                                           4, ctypes.c_void_p(st.cuda_stream)) == 0
-    v = y2.cpu().numpy()
-    assert np.all(v > 0) and np.all(v < 3e-38) and np.all(np.isfinite(v))
+    assert np.all(y2.cpu().numpy() == 0.0)
 
 
 def test_host_pipeline_matches_device_path(cuda_device):
