@@ -37,6 +37,13 @@
  *  - Launch failures return MF_ERR_CUDA. A fault the kernels detect while
  *    running (a pipeline wait that exceeded its time limit) is recorded on
  *    the device and reported by mf_get_device_error().
+ *  - libmfattn_checked.so, built from the same sources with -DMF_CHECKED,
+ *    exports the same calls. Its prologue, attention and backward kernels
+ *    compare every global index they compute with the extent of its buffer
+ *    before the access; an index outside records MF_ERR_BOUNDS (reported by
+ *    mf_get_device_error) and the access is skipped. The sub-layer's GEMM,
+ *    adaLN and table kernels are not checked. The product library,
+ *    libmfattn.so, compiles the checks away.
  */
 #ifndef MF_ATTN_H
 #define MF_ATTN_H
@@ -56,7 +63,9 @@ typedef enum {
   MF_ERR_WORKSPACE = -4,   /* workspace smaller than the *_workspace_bytes query  */
   MF_ERR_BUDGET = -5,      /* total tokens exceed the pack's token budget       */
   MF_ERR_CUDA = -6,        /* a CUDA runtime or driver call failed              */
-  MF_ERR_TIMEOUT = -7      /* a kernel pipeline wait ran out of time            */
+  MF_ERR_TIMEOUT = -7,     /* a kernel pipeline wait ran out of time            */
+  MF_ERR_BOUNDS = -8       /* checked build only: a kernel computed a global
+                              index outside its buffer (the access was skipped) */
 } mf_status;
 
 /* One packed sample: tokens [start, start + len) of the pack. 24 bytes. */
@@ -395,7 +404,8 @@ mf_status mf_selftest_timeout(int64_t limit_ns, void* stream);
 /*
  * Synchronises `stream`, then returns and clears the error the kernels
  * recorded on the current device since the last call (MF_OK if none,
- * MF_ERR_TIMEOUT if a pipeline wait ran out of time and the kernel gave up).
+ * MF_ERR_TIMEOUT if a pipeline wait ran out of time and the kernel gave up,
+ * MF_ERR_BOUNDS from the checked build's range checks).
  */
 mf_status mf_get_device_error(void* stream);
 

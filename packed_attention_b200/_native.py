@@ -6,6 +6,7 @@ the calls raise: there is no fallback path.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -14,6 +15,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmfattn.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libmfattn_checked.so")
 
 MF_TILE_M = 256
 MF_TILE_N = 128
@@ -21,6 +23,7 @@ MF_TILE_N = 128
 STATUS = {
     0: "MF_OK", -1: "MF_ERR_INVALID_ARG", -2: "MF_ERR_UNSUPPORTED", -3: "MF_ERR_ALIGNMENT",
     -4: "MF_ERR_WORKSPACE", -5: "MF_ERR_BUDGET", -6: "MF_ERR_CUDA", -7: "MF_ERR_TIMEOUT",
+    -8: "MF_ERR_BOUNDS",
 }
 
 
@@ -41,7 +44,8 @@ class WorkItem(ctypes.Structure):
 
 
 _lock = threading.Lock()
-_lib = None
+_libs = {}
+_use_checked = False
 
 P = ctypes.c_void_p
 I32 = ctypes.c_int32
@@ -81,21 +85,39 @@ SIGNATURES = {
 MF_STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
-def lib():
-    """The loaded library; raises if it has not been built."""
-    global _lib
+def _load(path):
     with _lock:
-        if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+        if path not in _libs:
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is missing: build it with "
                                    "`python -m packed_attention_b200.build`")
-            handle = ctypes.CDLL(LIB_PATH)
+            handle = ctypes.CDLL(path)
             for name, (res, args) in SIGNATURES.items():
                 f = getattr(handle, name)
                 f.restype = res
                 f.argtypes = args
-            _lib = handle
-    return _lib
+            _libs[path] = handle
+    return _libs[path]
+
+
+def lib():
+    """The loaded library (the checked build inside ``checked_build()``);
+    raises if it has not been built."""
+    return _load(CHECKED_LIB_PATH if _use_checked else LIB_PATH)
+
+
+@contextlib.contextmanager
+def checked_build():
+    """Route every call of the package through libmfattn_checked.so, the
+    build whose kernels range-check each global index they compute and
+    report a bad one as MF_ERR_BOUNDS (not thread-safe: for tests)."""
+    global _use_checked
+    prev = _use_checked
+    _use_checked = True
+    try:
+        yield _load(CHECKED_LIB_PATH)
+    finally:
+        _use_checked = prev
 
 
 def check(func: str, status: int):

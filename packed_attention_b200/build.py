@@ -2,7 +2,10 @@
 
 Run ``python -m packed_attention_b200.build`` (or call :func:`build`). The
 library is linked against the static CUDA runtime so it does not depend on
-which libcudart the host process already loaded.
+which libcudart the host process already loaded. ``build(checked=True)``
+builds libmfattn_checked.so from the same sources with -DMF_CHECKED: the
+kernels then range-check every global index they compute and report a bad
+one as MF_ERR_BOUNDS instead of accessing it.
 """
 from __future__ import annotations
 
@@ -15,6 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmfattn.so")
+CHECKED_LIB = os.path.join(HERE, "libmfattn_checked.so")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -29,24 +33,33 @@ def sources():
             os.path.join(CSRC, "plan.cpp")]
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = glob.glob(os.path.join(CSRC, "*")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = CHECKED_LIB if checked else LIB
+    if not force and not _stale(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, *sources()]
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc, *NVCC_FLAGS, *(["-DMF_CHECKED"] if checked else []),
+           *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, *sources()]
     subprocess.check_call(cmd, cwd=HERE)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force: bool = False) -> None:
+    """The product library and its checked twin."""
+    build(force=force)
+    build(force=force, checked=True)
 
 
 if __name__ == "__main__":
     print(build(force=True, verbose="-v" in sys.argv))
+    print(build(force=True, checked=True))

@@ -95,8 +95,9 @@ __device__ __forceinline__ void stage_put(uint32_t stage, int lane, int c, uint4
                : "memory");
 }
 
+// (buf, buf_bytes: the destination buffer, for the checked build's range check.)
 __device__ __forceinline__ void stage_flush(uint32_t stage, int lane, uint8_t* gbase, size_t stride,
-                                            int valid_rows) {
+                                            int valid_rows, const void* buf, size_t buf_bytes) {
   __syncwarp();
   const int q = lane & 3;
 #pragma unroll 1
@@ -107,7 +108,8 @@ __device__ __forceinline__ void stage_flush(uint32_t stage, int lane, uint8_t* g
                  : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
                  : "r"(stage + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4))
                  : "memory");
-    if (rr < valid_rows) *reinterpret_cast<uint4*>(gbase + rr * stride + q * 16) = o;
+    uint8_t* dst = gbase + rr * stride + q * 16;
+    if (rr < valid_rows && in_span(dst, 16, buf, buf_bytes)) *reinterpret_cast<uint4*>(dst) = o;
   }
   __syncwarp();
 }
@@ -115,6 +117,7 @@ __device__ __forceinline__ void stage_flush(uint32_t stage, int lane, uint8_t* g
 struct BwdParams {
   const mf_segment* segs;
   const mf_work_item* work;
+  int n_segs;
   const float* lse;       // [heads, total_tokens], natural log
   const float* delta;     // [heads, total_tokens]
   float* dhat;            // fp32 [total_tokens, heads, D]: dk_hat or dq_hat
@@ -213,7 +216,13 @@ __device__ __forceinline__ void bwd_producer(const BwdParams& p, BwdCtl& ctl, ui
   bool ok = true;
   for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
        idx = next_item(p.work, p.n_work, idx + stride, stride)) {
-    const ItemInfo it = load_item(p.segs, p.work, idx);
+    const ItemInfo it = load_item(p.segs, p.n_segs, p.work, idx);
+    // Tiles start inside the tensor (rows past T read as zeros).
+    if (kChecked) {
+      in_bounds(it.head, p.heads);
+      in_bounds(it.q0, p.total_tokens);
+      in_bounds(it.seg_start + it.seg_len - 1, p.total_tokens);
+    }
     const int passes = it.b_valid ? 2 : 1;
     for (int t = 0; t < passes && ok; ++t) {
       const int r0 = it.q0 + t * kSubM;
@@ -266,7 +275,7 @@ __device__ __forceinline__ void bwd_counts(const BwdParams& p, int& passes, int&
   const int stride = static_cast<int>(gridDim.x);
   for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work;
        idx = next_item(p.work, p.n_work, idx + stride, stride)) {
-    const ItemInfo it = load_item(p.segs, p.work, idx);
+    const ItemInfo it = load_item(p.segs, p.n_segs, p.work, idx);
     const int np = it.b_valid ? 2 : 1;
     passes += np;
     steps += np * it.n_kv;
@@ -327,7 +336,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool ok = true;
       for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
        idx = next_item(p.work, p.n_work, idx + stride, stride)) {
-        const ItemInfo it = load_item(p.segs, p.work, idx);
+        const ItemInfo it = load_item(p.segs, p.n_segs, p.work, idx);
         const int passes = it.b_valid ? 2 : 1;
         for (int t = 0; t < passes && ok; ++t) {
           const int n = it.n_kv;
@@ -393,7 +402,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
        idx = next_item(p.work, p.n_work, idx + stride, stride)) {
-      const ItemInfo it = load_item(p.segs, p.work, idx);
+      const ItemInfo it = load_item(p.segs, p.n_segs, p.work, idx);
       const int passes = it.b_valid ? 2 : 1;
       const int seg_end = it.seg_start + it.seg_len;
       const size_t stat0 = static_cast<size_t>(it.head) * p.total_tokens;
@@ -402,10 +411,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // (P = 0) and D = 0.
       auto load_stats = [&](int j, float& nl0, float& nl1, float& d0, float& d1) {
         const int q0 = it.seg_start + j * kBlockN + 64 * h + 2 * lane;
-        nl0 = q0 < seg_end ? -__ldg(p.lse + stat0 + q0) * kLog2e : -INFINITY;
-        nl1 = q0 + 1 < seg_end ? -__ldg(p.lse + stat0 + q0 + 1) * kLog2e : -INFINITY;
-        d0 = q0 < seg_end ? __ldg(p.delta + stat0 + q0) : 0.0f;
-        d1 = q0 + 1 < seg_end ? __ldg(p.delta + stat0 + q0 + 1) : 0.0f;
+        const long long n_stat = static_cast<long long>(p.heads) * p.total_tokens;
+        const bool in0 = q0 < seg_end && in_bounds(stat0 + q0, n_stat);
+        const bool in1 = q0 + 1 < seg_end && in_bounds(stat0 + q0 + 1, n_stat);
+        nl0 = in0 ? -__ldg(p.lse + stat0 + q0) * kLog2e : -INFINITY;
+        nl1 = in1 ? -__ldg(p.lse + stat0 + q0 + 1) * kLog2e : -INFINITY;
+        d0 = in0 ? __ldg(p.delta + stat0 + q0) : 0.0f;
+        d1 = in1 ? __ldg(p.delta + stat0 + q0 + 1) : 0.0f;
       };
       for (int t = 0; t < passes && ok; ++t, ++pc) {
         const int r0 = it.q0 + t * kSubM;
@@ -483,6 +495,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int tok0 = r0 + g4 * 32;  // token of this warp's first key row
         const int valid_rows = seg_end - tok0;
         const uint32_t stage = smem_addr(sStage) + warp * 2048;
+        // bytes of one fp32 [T, H, D] tensor (the bf16 dv is half of it)
+        const size_t rows_bytes = static_cast<size_t>(p.total_tokens) * p.heads * D * 4;
 #pragma unroll 1
         for (int c = 0; c < D / 64; ++c) {
           const int col = h * (D / 2) + 32 * c;
@@ -497,7 +511,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                  pack_bf16x2(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5])),
                                  pack_bf16x2(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7]))));
           stage_flush(stage, lane, reinterpret_cast<uint8_t*>(p.dv + orow0),
-                      static_cast<size_t>(p.heads) * D * 2, valid_rows);
+                      static_cast<size_t>(p.heads) * D * 2, valid_rows, p.dv, rows_bytes / 2);
           tmem_ld32_sync(tmem + lane_off + kColDK + col, r);
 #pragma unroll
           for (int k2 = 0; k2 < 2; ++k2) {
@@ -511,7 +525,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                    __float_as_uint(__uint_as_float(r[e + 3]) * p.scale)));
             }
             stage_flush(stage, lane, reinterpret_cast<uint8_t*>(p.dhat + orow0 + 16 * k2),
-                        static_cast<size_t>(p.heads) * D * 4, valid_rows);
+                        static_cast<size_t>(p.heads) * D * 4, valid_rows, p.dhat, rows_bytes);
           }
         }
         tc_fence_before_sync();
@@ -583,7 +597,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool ok = true;
       for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
        idx = next_item(p.work, p.n_work, idx + stride, stride)) {
-        const ItemInfo it = load_item(p.segs, p.work, idx);
+        const ItemInfo it = load_item(p.segs, p.n_segs, p.work, idx);
         const int passes = it.b_valid ? 2 : 1;
         for (int t = 0; t < passes && ok; ++t) {
           const int n = it.n_kv;
@@ -651,7 +665,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
        idx = next_item(p.work, p.n_work, idx + stride, stride)) {
-      const ItemInfo it = load_item(p.segs, p.work, idx);
+      const ItemInfo it = load_item(p.segs, p.n_segs, p.work, idx);
       const int passes = it.b_valid ? 2 : 1;
       const int seg_end = it.seg_start + it.seg_len;
       for (int t = 0; t < passes && ok; ++t, ++pc) {
@@ -667,8 +681,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t qv[D / 4], ov[D / 4];
 #pragma unroll
           for (int v = 0; v < kV; ++v) {
-            const uint4 a = q < p.total_tokens ? __ldg(p.q_rows + base + v) : make_uint4(0, 0, 0, 0);
-            const uint4 b = q < p.total_tokens ? __ldg(p.do_rows + base + v) : make_uint4(0, 0, 0, 0);
+            const bool in = q < p.total_tokens &&
+                            in_bounds(base + v, static_cast<long long>(p.total_tokens) * p.heads * (D / 8));
+            const uint4 a = in ? __ldg(p.q_rows + base + v) : make_uint4(0, 0, 0, 0);
+            const uint4 b = in ? __ldg(p.do_rows + base + v) : make_uint4(0, 0, 0, 0);
             qv[4 * v] = a.x; qv[4 * v + 1] = a.y; qv[4 * v + 2] = a.z; qv[4 * v + 3] = a.w;
             ov[4 * v] = b.x; ov[4 * v + 1] = b.y; ov[4 * v + 2] = b.z; ov[4 * v + 3] = b.w;
           }
@@ -684,8 +700,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (lane == 0) mbar_arrive(&ctl.q_ready);
         }
         const size_t si = static_cast<size_t>(it.head) * p.total_tokens + q;
-        const float nl = row_in ? -__ldg(p.lse + si) * kLog2e : 0.0f;
-        const float drow = row_in ? __ldg(p.delta + si) : 0.0f;
+        const bool stat_in = row_in && in_bounds(si, static_cast<long long>(p.heads) * p.total_tokens);
+        const float nl = stat_in ? -__ldg(p.lse + si) * kLog2e : 0.0f;
+        const float drow = stat_in ? __ldg(p.delta + si) : 0.0f;
         const uint64_t nl2 = f32x2(nl, nl), d2 = f32x2(drow, drow);
         for (int j = 0; j < it.n_kv; ++j) {
           if (!warp_wait_bar(&ctl.s_full, ns & 1, abort_flag)) { ok = false; break; }
@@ -742,6 +759,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int tok0 = r0 + g4 * 32;  // token of this warp's first query row
         const int valid_rows = seg_end - tok0;
         const uint32_t stage = smem_addr(sStage) + warp * 2048;
+        // bytes of one fp32 [T, H, D] tensor (the bf16 dv is half of it)
+        const size_t rows_bytes = static_cast<size_t>(p.total_tokens) * p.heads * D * 4;
 #pragma unroll 1
         for (int c = 0; c < D / 64; ++c) {
           const int col = h * (D / 2) + 32 * c;
@@ -760,7 +779,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                    __float_as_uint(__uint_as_float(r[e + 3]) * p.scale)));
             }
             stage_flush(stage, lane, reinterpret_cast<uint8_t*>(p.dhat + orow0 + 16 * k2),
-                        static_cast<size_t>(p.heads) * D * 4, valid_rows);
+                        static_cast<size_t>(p.heads) * D * 4, valid_rows, p.dhat, rows_bytes);
           }
         }
         tc_fence_before_sync();

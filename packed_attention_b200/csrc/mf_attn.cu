@@ -267,6 +267,7 @@ mf_status packed_attention_impl(const void* v, const mf_segment* segs_dev, int32
   mf::AttnParams prm;
   prm.segs = segs_dev;
   prm.work = work_dev;
+  prm.n_segs = n_samples;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
   prm.n_work = n_work;
@@ -486,6 +487,7 @@ extern "C" mf_status mf_joint_attn_bwd(
   mf::BwdParams prm;
   prm.segs = segs_dev;
   prm.work = work_dev;
+  prm.n_segs = n_samples;
   prm.lse = lse;
   prm.delta = delta;
   prm.dv = static_cast<__nv_bfloat16*>(dv);

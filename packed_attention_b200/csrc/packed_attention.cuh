@@ -68,11 +68,10 @@
 #include <cstdint>
 
 #include "../../include/mf_attn.h"
+#include "bounds.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mf {
-
-__device__ int32_t g_device_error;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms for in-flight work on abort
@@ -114,6 +113,7 @@ struct AttnConfig {
 struct AttnParams {
   const mf_segment* segs;
   const mf_work_item* work;
+  int n_segs;
   __nv_bfloat16* out;
   float* lse;        // optional [heads, total_tokens]: natural-log softmax normaliser per row
   int n_work;
@@ -131,10 +131,13 @@ struct ItemInfo {
   bool b_valid;
 };
 
-__device__ __forceinline__ ItemInfo load_item(const mf_segment* segs, const mf_work_item* work,
-                                              int idx) {
+// (A work item naming a segment outside [0, n_segs) is a caller error: the
+// checked build records it and uses segment 0 instead, so that every role of
+// the kernel still walks the same items.)
+__device__ __forceinline__ ItemInfo load_item(const mf_segment* segs, int n_segs,
+                                              const mf_work_item* work, int idx) {
   const mf_work_item wi = work[idx];
-  const mf_segment sg = segs[wi.seg];
+  const mf_segment sg = segs[in_bounds(wi.seg, n_segs) ? wi.seg : 0];
   ItemInfo it;
   it.seg_start = sg.start;
   it.seg_len = sg.len;
@@ -146,7 +149,7 @@ __device__ __forceinline__ ItemInfo load_item(const mf_segment* segs, const mf_w
 }
 
 __device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int idx) {
-  return load_item(p.segs, p.work, idx);
+  return load_item(p.segs, p.n_segs, p.work, idx);
 }
 
 // The first work-list position >= idx in this CTA's stride that holds an
@@ -183,7 +186,7 @@ __device__ __forceinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volati
     if (global_timer_ns() - t0 > limit_ns) {
       if (abort_flag) {
         *abort_flag = 1;
-        atomicCAS(&g_device_error, 0, static_cast<int32_t>(MF_ERR_TIMEOUT));
+        record_error(MF_ERR_TIMEOUT);
       }
       return false;
     }
@@ -301,6 +304,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
            idx = next_item(p.work, p.n_work, idx + stride, stride), ++k) {
         const ItemInfo it = load_item(p, idx);
+        // Tiles start inside the tensor (a tile may run past its end: TMA
+        // fills the rows past T with zeros).
+        if (kChecked) {
+          in_bounds(it.head, p.heads);
+          in_bounds(it.q0, p.total_tokens);
+          in_bounds(it.seg_start + it.seg_len - 1, p.total_tokens);
+        }
         if (k > 0 && !wait_bar(&ctl.q_empty, (k - 1) & 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(&ctl.q_full, 2 * kTile);
 #pragma unroll
@@ -520,9 +530,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float inv_l = 1.0f / l;
       // log of the row's softmax normaliser, sum_u exp(s_u * scale), for the
       // backward pass: m and l are in the exp2 domain of s * scale * log2(e).
-      if (p.lse && row_in)
-        p.lse[static_cast<size_t>(it.head) * p.total_tokens + q_row] =
-            (m + log2f(l)) * 0.6931471805599453f;
+      if (p.lse && row_in) {
+        const size_t li = static_cast<size_t>(it.head) * p.total_tokens + q_row;
+        if (in_bounds(li, static_cast<long long>(p.heads) * p.total_tokens))
+          p.lse[li] = (m + log2f(l)) * 0.6931471805599453f;
+      }
       // O / l in 64-dim halves through this warp's 4 KB of shared memory:
       // each lane writes its row (128 bytes, 16-byte chunk c at c ^ (row % 8)),
       // then each store instruction of the warp writes four whole 128-byte row
@@ -555,9 +567,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int rr = 4 * i + rr0;
           const uint4 o = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((cc ^ (rr & 7)) << 4));
           const int tok = row0 + rr;
-          if (tok < row_end)
-            reinterpret_cast<uint4*>(p.out)[(static_cast<size_t>(tok) * p.heads + it.head) * (D / 8) +
-                                            8 * half + cc] = o;
+          const size_t oi = (static_cast<size_t>(tok) * p.heads + it.head) * (D / 8) + 8 * half + cc;
+          if (tok < row_end &&
+              in_bounds(oi, static_cast<long long>(p.total_tokens) * p.heads * (D / 8)))
+            reinterpret_cast<uint4*>(p.out)[oi] = o;
         }
         __syncwarp();
       }

@@ -33,6 +33,7 @@ extern "C" const char* mf_status_string(mf_status status) {
     case MF_ERR_BUDGET: return "MF_ERR_BUDGET";
     case MF_ERR_CUDA: return "MF_ERR_CUDA";
     case MF_ERR_TIMEOUT: return "MF_ERR_TIMEOUT";
+    case MF_ERR_BOUNDS: return "MF_ERR_BOUNDS";
   }
   return "MF_ERR_UNKNOWN";
 }

@@ -30,6 +30,7 @@
 #include <cstdint>
 
 #include "../../include/mf_attn.h"
+#include "bounds.cuh"
 
 namespace mf {
 
@@ -131,12 +132,14 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
 
   const float inv_d = 1.0f / D;
   const size_t row0 = static_cast<size_t>(t) * heads * kVecPerRow + vec;
+  const long long n_vec = static_cast<long long>(total_tokens) * heads * kVecPerRow;
 #pragma unroll 2
   for (int h = 0; h < heads; ++h) {
     const size_t idx = row0 + static_cast<size_t>(h) * kVecPerRow;
+    const bool in = in_bounds(idx, n_vec);
     float xq[8], xk[8];
-    unpack8(__ldg(q + idx), xq);
-    unpack8(__ldg(k + idx), xk);
+    unpack8(in ? __ldg(q + idx) : make_uint4(0, 0, 0, 0), xq);
+    unpack8(in ? __ldg(k + idx) : make_uint4(0, 0, 0, 0), xk);
     float ssq = 0.f, ssk = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_kernel(
       yk[2 * i] = ka * cs[i] - kb * sn[i];
       yk[2 * i + 1] = ka * sn[i] + kb * cs[i];
     }
-    if (active) {
+    if (active && in) {
       q_hat[idx] = pack8(yq);
       k_hat[idx] = pack8(yk);
     }

@@ -37,17 +37,21 @@ __global__ void __launch_bounds__(kPrologueThreads) bwd_delta_kernel(
   const bool active = t_raw < total_tokens;
   const int t = active ? t_raw : total_tokens - 1;
   const size_t row0 = static_cast<size_t>(t) * heads * kVecPerRow + vec;
+  const long long n_vec = static_cast<long long>(total_tokens) * heads * kVecPerRow;
   for (int h = 0; h < heads; ++h) {
     const size_t idx = row0 + static_cast<size_t>(h) * kVecPerRow;
+    const bool in = in_bounds(idx, n_vec);
     float a[8], b[8];
-    unpack8(__ldg(out + idx), a);
-    unpack8(__ldg(dout + idx), b);
+    unpack8(in ? __ldg(out + idx) : make_uint4(0, 0, 0, 0), a);
+    unpack8(in ? __ldg(dout + idx) : make_uint4(0, 0, 0, 0), b);
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) s = fmaf(a[i], b[i], s);
 #pragma unroll
     for (int o = kVecPerRow / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, kVecPerRow);
-    if (active && vec == 0) delta[static_cast<size_t>(h) * total_tokens + t] = s;
+    const size_t di = static_cast<size_t>(h) * total_tokens + t;
+    if (active && vec == 0 && in_bounds(di, static_cast<long long>(heads) * total_tokens))
+      delta[di] = s;
   }
 }
 
@@ -140,15 +144,18 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_bwd_kernel(
 
   const float inv_d = 1.0f / D;
   const size_t row0 = static_cast<size_t>(t) * heads * kVecPerRow + vec;
+  const long long n_vec = static_cast<long long>(total_tokens) * heads * kVecPerRow;
 #pragma unroll 1
   for (int h = 0; h < heads; ++h) {
     const size_t idx = row0 + static_cast<size_t>(h) * kVecPerRow;
+    const bool in = in_bounds(idx, n_vec);  // covers dq_hat / dk_hat's 2 * idx + 1 too
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
       float x[8], dy[8];
-      unpack8(__ldg((which ? k : q) + idx), x);
+      unpack8(in ? __ldg((which ? k : q) + idx) : make_uint4(0, 0, 0, 0), x);
       const float4* dh = which ? dk_hat : dq_hat;
-      const float4 d0 = __ldg(dh + 2 * idx), d1 = __ldg(dh + 2 * idx + 1);
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 d0 = in ? __ldg(dh + 2 * idx) : z4, d1 = in ? __ldg(dh + 2 * idx + 1) : z4;
       const float dx_hat[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
       // transposed rotation: (a, b) -> (a cos + b sin, -a sin + b cos)
 #pragma unroll
@@ -179,7 +186,7 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_bwd_kernel(
       float y[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) y[i] = r * fmaf(-xn[i], c, dxn[i]);
-      if (active) (which ? dk : dq)[idx] = pack8(y);
+      if (active && in) (which ? dk : dq)[idx] = pack8(y);
     }
   }
 
@@ -198,7 +205,8 @@ __global__ void __launch_bounds__(kPrologueThreads) qk_prologue_bwd_kernel(
     float s = 0.f;
     for (int tk = 0; tk < kTokPerBlock; ++tk)
       if (s_text[tk] == want_text) s += s_red[tk][which][m];
-    partial[static_cast<size_t>(blockIdx.x) * 4 * D + o] = s;
+    const size_t pi = static_cast<size_t>(blockIdx.x) * 4 * D + o;
+    if (in_bounds(pi, static_cast<long long>(gridDim.x) * 4 * D)) partial[pi] = s;
   }
 }
 
@@ -217,7 +225,10 @@ __global__ void __launch_bounds__(32 * kReduceWarps) dgamma_reduce_kernel(
   const int b0 = w * per, b1 = min(n_blocks, b0 + per);
   float s = 0.f;
   if (o < n_out)
-    for (int b = b0; b < b1; ++b) s += __ldg(partial + static_cast<size_t>(b) * n_out + o);
+    for (int b = b0; b < b1; ++b) {
+      const size_t pi = static_cast<size_t>(b) * n_out + o;
+      if (in_bounds(pi, static_cast<long long>(n_blocks) * n_out)) s += __ldg(partial + pi);
+    }
   s_part[w][lane] = s;
   __syncthreads();
   if (w == 0 && o < n_out) {

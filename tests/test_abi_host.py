@@ -59,6 +59,18 @@ def test_header_declares_the_documented_calls():
     assert header_functions() == DOCUMENTED_ABI
 
 
+def test_checked_build_exports_the_same_calls():
+    """libmfattn_checked.so (-DMF_CHECKED) exports every declared call and
+    knows the status its range checks report."""
+    build(checked=True)
+    with _native.checked_build() as checked:
+        for n in header_functions():
+            assert hasattr(checked, n), n
+        assert checked.mf_status_string(-8).decode() == "MF_ERR_BOUNDS"
+        assert _native.lib() is checked
+    assert _native.lib() is not checked
+
+
 def test_status_strings(lib):
     assert lib.mf_abi_version() == 4
     for code, name in _native.STATUS.items():

@@ -4,16 +4,24 @@ Inputs are the same seeded bf16 tensors for both sides; dL/dout is a seeded
 bf16 tensor. The GPU path recomputes q_hat, k_hat, takes P from the forward's
 log-normaliser, rounds P and dS to bf16 for the tensor cores and the
 gradients once to bf16 at the end; the oracle differentiates the fp64
-forward exactly. Tolerance (relative RMS over all elements of a gradient,
-and max-abs over the gradient's RMS): each gradient passes through about
-three bf16 roundings (2^-9 relative each: q_hat / k_hat or P, dS, the output)
-and sums of ~L terms of random sign, so the relative RMS error sits near
-3 * 2^-9 / sqrt(3) ~ 3.4e-3 (measured: 3.2e-3 to 4.9e-3); the bound is 1e-2.
-An element's error scales with the element, and the largest elements reach
-~5x the RMS with up to ~2^-7 relative error where a sum has few terms (a
-6-token sample), so max-abs is bounded by 0.25 of the gradient's RMS
-(measured: up to 0.12). A gamma of a modality the pack does not contain has
-an exactly zero gradient on both sides.
+forward exactly.
+
+Error model, fixed before measuring (the bounds below follow from it):
+* every gradient element is a sum, over the tokens of its sample, of
+  products that went through three bf16 roundings (q_hat / k_hat, P, dS),
+  each a relative error of at most 2^-9 (uniform: RMS 2^-9 / sqrt(3));
+* the terms have random signs, so the intermediate error of one element is
+  Gaussian with an RMS of at most sigma = 3 * 2^-9 / sqrt(3) ~ 3.4e-3 (the
+  three added linearly, their worst correlation) times the scale rho of the
+  element's row: the RMS of the reference gradient over its (token, head)
+  row, or over the whole vector for a gamma gradient (errors are relative to
+  the row, since the norm backward scales each row by its own 1 / rms);
+* then the element is rounded once to bf16, at most 2^-8 of the value.
+Hence, per element, |got - ref| <= 2^-8 (|ref| + E) + E with E = 8 sigma rho
+(a Gaussian passes 8 sigma with probability ~1e-15; fewer than 1e7 elements
+are tested), and over all elements a relative RMS error <= 1e-2 (~3 sigma).
+A gamma of a modality the pack does not contain has an exactly zero gradient
+on both sides.
 """
 import json
 import os
@@ -32,7 +40,8 @@ from test_gpu_parity import bf16_to_f64, to_dev
 pytestmark = pytest.mark.gpu
 
 REL_RMS_BWD = 1e-2
-MAX_ABS_REL_BWD = 0.25
+SIGMA_BWD = 3 * 2.0 ** -9 / np.sqrt(3)  # model RMS of the intermediate error, per unit of rho
+K_SIGMA = 8.0
 NAMES = pa.GAMMA_NAMES
 
 
@@ -41,12 +50,30 @@ def dout_bits(w: Workload):
     return synth.f64_to_bf16_bits(z.reshape(w.total_tokens, w.heads, w.head_dim))
 
 
-def rel_errors(got, ref):
-    diff = got - ref
+def elementwise_bound(ref, per_row):
+    """|got - ref| allowed per element by the error model above: rho is the
+    RMS of ref over the last axis (per_row) or over everything."""
+    axis = -1 if per_row else None
+    rho = np.sqrt(np.mean(ref ** 2, axis=axis, keepdims=per_row))
+    e = K_SIGMA * SIGMA_BWD * rho
+    return np.ldexp(np.abs(ref) + e, -8) + e
+
+
+def grad_errors(got, ref, per_row):
+    """(fraction of the element-wise bound used at worst, relative RMS error,
+    largest error per head over the head's RMS) for one gradient."""
+    diff = np.abs(got - ref)
+    bound = elementwise_bound(ref, per_row)
+    used = float(np.max(np.where(bound > 0, diff / np.where(bound > 0, bound, 1.0),
+                                 np.where(diff > 0, np.inf, 0.0))))
     rms = float(np.sqrt(np.mean(ref ** 2)))
-    if rms == 0.0:  # nothing contributes: both sides must be exactly zero
-        return (0.0, 0.0) if not np.any(got) else (float("inf"), float("inf"))
-    return float(np.max(np.abs(diff))) / rms, float(np.sqrt(np.mean(diff ** 2))) / rms
+    rel_rms = float(np.sqrt(np.mean(diff ** 2))) / rms if rms > 0 else (
+        0.0 if not np.any(got) else float("inf"))
+    heads = None
+    if ref.ndim == 3:
+        heads = [float(np.max(diff[:, h]) / max(np.sqrt(np.mean(ref[:, h] ** 2)), 1e-300))
+                 for h in range(ref.shape[1])]
+    return used, rel_rms, heads
 
 
 def report(name, errs):
@@ -82,13 +109,14 @@ def check_grads(name, g, ref, heads=None, gammas=True):
     errs = {}
     for key in ("dq", "dk", "dv"):
         got = bf16_to_f64(g[key])[:, sel]
-        errs[key] = rel_errors(got, ref[key])
+        errs[key] = grad_errors(got, ref[key], per_row=True)
     if gammas:
         for n in NAMES:
-            errs[n] = rel_errors(g[n].double().cpu().numpy(), ref["dgamma"][n])
-    report(name, errs)
-    for key, (mx, rr) in errs.items():
-        assert rr <= REL_RMS_BWD and mx <= MAX_ABS_REL_BWD, (key, mx, rr)
+            errs[n] = grad_errors(g[n].double().cpu().numpy(), ref["dgamma"][n], per_row=False)
+    report(name, {k: {"bound_used": u, "rel_rms": r, "head_max_over_rms": hd}
+                  for k, (u, r, hd) in errs.items()})
+    for key, (used, rr, _) in errs.items():
+        assert rr <= REL_RMS_BWD and used <= 1.0, (key, used, rr)
 
 
 SMALL = [
