@@ -145,6 +145,10 @@ struct BwdCtl {
 
 // D (+)= A (TMEM, bf16: 128 lanes x 128 K, K 0..63 in columns [0,32) and
 // K 64..127 in [64,96)) * B (shared, MN-major [K = 128 rows][N = D]).
+// Low half of a shared-memory descriptor made by smem_desc_sw128(.., .., 1024),
+// whose high half is kDescHiSw128, for issue_qk.
+__device__ __forceinline__ uint32_t lo32(uint64_t desc) { return static_cast<uint32_t>(desc); }
+
 template <int D>
 __device__ __forceinline__ void issue_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                              bool accumulate) {
@@ -344,11 +348,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after_sync();
           if (!wait_bar(&ctl.x_full[g % NX], (g / NX) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_qk<D>(tmem + kColS, k_desc, x_k + (g % NX) * kStep);
+          issue_qk<D>(tmem + kColS, lo32(k_desc), lo32(x_k + (g % NX) * kStep));
           mma_commit(&ctl.s_full);
           if (!wait_bar(&ctl.y_full[g % NY], (g / NY) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_qk<D>(tmem + kColDP, v_desc, y_k + (g % NY) * kStep);
+          issue_qk<D>(tmem + kColDP, lo32(v_desc), lo32(y_k + (g % NY) * kStep));
           mma_commit(&ctl.dp_full);
           for (int j = 0; j < n && ok; ++j) {
             const int gj = g + j, gn = gj + 1;
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (more) {
               if (!wait_bar(&ctl.x_full[gn % NX], (gn / NX) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
-              issue_qk<D>(tmem + kColS, k_desc, x_k + (gn % NX) * kStep);
+              issue_qk<D>(tmem + kColS, lo32(k_desc), lo32(x_k + (gn % NX) * kStep));
               mma_commit(&ctl.s_full);
             }
             if (!wait_bar(&ctl.ds_ready, nph & 1, abort_flag)) { ok = false; break; }
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (more) {
               if (!wait_bar(&ctl.y_full[gn % NY], (gn / NY) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
-              issue_qk<D>(tmem + kColDP, v_desc, y_k + (gn % NY) * kStep);
+              issue_qk<D>(tmem + kColDP, lo32(v_desc), lo32(y_k + (gn % NY) * kStep));
               mma_commit(&ctl.dp_full);
             }
           }

@@ -133,39 +133,7 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ cu_seqlens,
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= total_tokens * (D / 2)) return;
   const int t = idx / (D / 2), pair = idx % (D / 2);
-  int lo = 0, hi = n_samples;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(cu_seqlens + mid) <= t) lo = mid; else hi = mid;
-  }
-  const int j = t - __ldg(&segs[lo].start);
-  const int n_text = __ldg(&segs[lo].n_text);
-  if (j < n_text) {
-    table[idx] = make_float2(1.0f, 0.0f);
-    return;
-  }
-  const int gw = __ldg(&segs[lo].grid_w);
-  const int hw = __ldg(&segs[lo].grid_h) * gw;
-  const int spatial = (D - frame_dims) / 2;
-  const int frame = (j - n_text) / hw, p = (j - n_text) % hw;
-  const int e = 2 * pair;
-  int pos, first, width;
-  if (e < frame_dims) {
-    pos = frame; first = 0; width = frame_dims;
-  } else if (e < frame_dims + spatial) {
-    pos = p / gw; first = frame_dims; width = spatial;
-  } else {
-    pos = p % gw; first = frame_dims + spatial; width = spatial;
-  }
-  constexpr double kLog2Base = 13.287712379549449;
-  constexpr double kTwoPi = 6.283185307179586;
-  constexpr double kInvTwoPi = 0.15915494309189535;
-  const double theta = exp2(-(2.0 * ((e - first) / 2) / width) * kLog2Base);
-  double ang = static_cast<double>(pos) * theta;
-  ang -= kTwoPi * rint(ang * kInvTwoPi);
-  float sn, cs;
-  sincosf(static_cast<float>(ang), &sn, &cs);
-  table[idx] = make_float2(cs, sn);
+  table[idx] = pair_cos_sin<D>(token_position(cu_seqlens, segs, n_samples, t), pair, frame_dims);
 }
 
 // Per 128-row tile: bit 0 if it holds text tokens, bit 1 if image tokens.

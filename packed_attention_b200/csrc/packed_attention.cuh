@@ -20,23 +20,33 @@
 //                    (bf16) back into TMEM over S, and rescale O in TMEM only
 //                    when the running max of a row inside the sample grew by
 //                    more than 2^8 (a stale max keeps p <= 256: exact enough
-//                    in bf16, safe in fp32). At the end of an item: O / l ->
+//                    in bf16, safe in fp32). At the end of an item a thread
+//                    stores its row's log-normaliser (when asked), hands 1/l
+//                    to the epilogue warps and goes straight on to the next
+//                    item's first S.
+//   warps 8-11       epilogue, one warp per TMEM lane quarter (32 rows of
+//                    each sub-tile): after an item's last PV_t, O_t / l ->
 //                    bf16 rows through 4 KB of shared memory per warp, so
-//                    that the stores write whole 128-byte row segments,
-//                    skipping rows past the sample end.
-//   warp 8 (1 lane)  TMA producer: both Q sub-tiles per item, then K_j, V_j
+//                    that the stores write whole 128-byte row segments
+//                    (rows past the sample end are not stored); then O_t is
+//                    free for the next item's first PV_t.
+//   warp 12 (1 lane) TMA producer: both Q sub-tiles per item, then K_j, V_j
 //                    into a ring of shared-memory stages (128-byte swizzled
 //                    boxes of 128 rows x 64 dims).
-//   warps 10-11      idle; they complete warpgroup 2 so that its registers
-//                    can be handed to the softmax warpgroups (setmaxnreg:
-//                    softmax 200 per thread, warpgroup 2 96 per thread).
-//   warp 9 (1 lane)  MMA issuer (also owns the TMEM allocation):
+//   warp 13 (1 lane) MMA issuer (also owns the TMEM allocation), one stream
+//                    across item boundaries:
 //                      S_a(0) S_b(0) | PV_a(j) S_a(j+1) PV_b(j) S_b(j+1) | ...
+//                    where after an item's last step "j+1" is the next item's
+//                    step 0, so its first S and softmax overlap the epilogue.
 //                    S = Q K^T with both operands in shared memory; O += P V
 //                    with P from TMEM and V (an MN-major operand) from shared
 //                    memory; fp32 accumulators in TMEM. While softmax a works
 //                    on S_a(j+1) the tensor core runs PV_b(j) and S_b(j+1),
 //                    and the other way round.
+//   warps 14-15      idle; with warps 12-13 they form warpgroup 3, which
+//                    (like the epilogue warpgroup) gives registers to the
+//                    softmax warpgroups (setmaxnreg: softmax 184 per thread,
+//                    epilogue 64, producer and MMA 80).
 //
 // TMEM (512 columns): S_a [0,128) O_a [128,256) S_b [256,384) O_b [384,512).
 // P_t(j) overwrites the first 64 columns of S_t after the softmax has read
@@ -54,7 +64,10 @@
 //   p_half[t][h]       softmax t (4 warps) -> MMA, one phase per half (64
 //                      keys) of P_t: the first half of PV_t starts while the
 //                      softmax computes the second half's exponentials
-//   o_ready[t]         MMA -> softmax t after the item's last PV_t
+//   o_ready[t]         MMA -> epilogue after an item's last PV_t
+//   stat_ready[t]      softmax t (128 threads) -> epilogue: 1/l of each row
+//   o_free[t]          epilogue (4 warps) -> MMA: O_t drained; the next
+//                      item's first PV_t (which overwrites O_t) may go
 //
 // Every wait is bounded (kWaitLimitNs). A wait that runs out records
 // MF_ERR_TIMEOUT in the device error word and raises the CTA's abort flag;
@@ -75,15 +88,20 @@ namespace mf {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms for in-flight work on abort
-constexpr int kAttnThreads = 384;
-constexpr uint32_t kSoftmaxRegs = 200;   // per thread, warpgroups 0 and 1
-constexpr uint32_t kControlRegs = 96;    // per thread, warpgroup 2
-// The split must fit in what the CTA is launched with (384 x regs/thread):
+constexpr int kAttnThreads = 512;
+constexpr uint32_t kSoftmaxRegs = 184;   // per thread, warpgroups 0 and 1
+constexpr uint32_t kEpilogueRegs = 64;   // per thread, warpgroup 2
+constexpr uint32_t kControlRegs = 80;    // per thread, warpgroup 3
+// The split must fit in what the CTA is launched with (512 x regs/thread):
 // the host refuses to launch if the compiled kernel uses fewer registers.
-constexpr int kMinLaunchRegs = (2 * 128 * kSoftmaxRegs + 128 * kControlRegs + kAttnThreads - 1) /
-                               kAttnThreads;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMinLaunchRegs =
+    (2 * 128 * kSoftmaxRegs + 128 * kEpilogueRegs + 128 * kControlRegs + kAttnThreads - 1) /
+    kAttnThreads;
+static_assert(2 * kSoftmaxRegs + kEpilogueRegs + kControlRegs <= 4 * 128,
+              "the warpgroups' registers must fit the 64K register file");
+constexpr int kEpilogueWarp0 = 8;  // warps 8-11
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr int kSubM = 128;             // rows of one query sub-tile (MMA M)
 constexpr int kBlockN = MF_TILE_N;     // keys per step (MMA N of S, K of PV)
 constexpr int kBoxBytes = 128 * 128;   // 128 rows x 64 bf16 = one 128-byte swizzle span
@@ -102,9 +120,9 @@ struct AttnConfig {
   static constexpr int kTileBytes = kSubM * D * 2;  // one 128-row tile of Q, K or V
   // Deep enough that each K/V load is requested a full key step before use.
   static constexpr int kStages = D == 128 ? 4 : 6;
-  // Per softmax warp: 32 output rows x 64 dims (bf16) staged for coalesced
+  // Per epilogue warp: 32 output rows x 64 dims (bf16) staged for coalesced
   // stores at the end of an item.
-  static constexpr int kStageBytes = 8 * 32 * 128;
+  static constexpr int kStageBytes = 4 * 32 * 128;
   static constexpr int kSmemBytes = kTileBytes * (2 + kStages) + kStageBytes + 1024;
   static_assert(kStages <= kMaxStages, "ring too deep");
   static_assert(kSmemBytes <= 226 * 1024, "over the 227 KB of shared memory a CTA may use");
@@ -168,7 +186,10 @@ struct SharedCtl {
   uint64_t s_full[2];
   uint64_t p_half[2][2];  // first / second 64 keys of P_t
   uint64_t o_ready[2];
+  uint64_t stat_ready[2];
+  uint64_t o_free[2];
   uint64_t drain;
+  float inv_l[2][kSubM];  // 1 / l of each row of the item that just ended, per sub-tile
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -215,13 +236,14 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
 // S (tmem) = Q (smem) K^T (smem): M=128, N=128, K=D in steps of 16. Both are
 // K-major with the 128-byte swizzle: a K step of 16 elements is 32 bytes
 // inside a 128-byte row; 64-element column blocks are one box apart.
+// (Descriptors by their low 32 bits, see mma_ss_lo.)
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
   constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, kBlockN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint64_t off = static_cast<uint64_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4);
-    mma_ss(d_tmem, q_desc + off, k_desc + off, kIdesc, kk > 0 ? 1u : 0u);
+    const uint32_t off = static_cast<uint32_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4);
+    mma_ss_lo(d_tmem, q_lo + off, k_lo + off, kIdesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -230,13 +252,13 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint6
 // keys are two 8-row swizzle atoms (2 KB); 64-dim blocks are one box apart
 // (the descriptor's leading byte offset).
 template <int D, int k0, int k1>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc,
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo,
                                          bool accumulate) {
   constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, D, 0, 1);
 #pragma unroll
   for (int kk = k0; kk < k1; ++kk)
-    mma_ts(o_tmem, p_tmem + kk * 8, v_desc + static_cast<uint64_t>(kk * (2048 >> 4)), kIdesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_lo(o_tmem, p_tmem + kk * 8, v_lo + static_cast<uint32_t>(kk * (2048 >> 4)), kIdesc,
+              (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -254,7 +276,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;                // sub-tile a, then sub-tile b
   uint8_t* sKV = smem + 2 * kTile;   // NS stages
-  uint8_t* sOut = sKV + NS * kTile;  // output staging, 4 KB per softmax warp
+  uint8_t* sOut = sKV + NS * kTile;  // output staging, 4 KB per epilogue warp
   volatile int32_t* abort_flag = &ctl.abort;
 
   const int warp = threadIdx.x / 32;
@@ -272,6 +294,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&ctl.p_half[t][0], 4);
       mbar_init(&ctl.p_half[t][1], 4);
       mbar_init(&ctl.o_ready[t], 1);
+      mbar_init(&ctl.stat_ready[t], kSubM);
+      mbar_init(&ctl.o_free[t], 4);
     }
     mbar_init(&ctl.drain, 1);
     ctl.abort = 0;
@@ -291,10 +315,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = ctl.tmem_base;
   const int stride = static_cast<int>(gridDim.x);
-  if (warp >= 8) {
-    // Warpgroup 2 (producer, MMA issuer, two idle warps) gives registers away.
+  // Each warpgroup re-splits its registers first thing in its own branch, so
+  // that the code of every role is compiled under its own budget:
+  // warpgroup 3 (producer, MMA issuer, two idle warps) and warpgroup 2
+  // (epilogue) give registers to warpgroups 0 and 1 (softmax).
+  if (warp >= 12) {
     setmaxnreg_dec<kControlRegs>();
-  }
   if (warp == kProducerWarp) {
     // ------------------------------------------------------ TMA producer ---
     if (lane == 0) {
@@ -342,81 +368,115 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------- MMA issuer ---
     if (lane == 0) {
-      const uint64_t q_desc[2] = {smem_desc_sw128(smem_addr(sQ), 16, 1024),
-                                  smem_desc_sw128(smem_addr(sQ + kTile), 16, 1024)};
+      const uint32_t q_desc[2] = {smem_desc_sw128_lo(smem_addr(sQ), 16),
+                                  smem_desc_sw128_lo(smem_addr(sQ + kTile), 16)};
       // K stages as K-major operands, V stages as MN-major operands.
-      const uint64_t k_desc0 = smem_desc_sw128(smem_addr(sKV), 16, 1024);
-      const uint64_t v_desc0 = smem_desc_sw128(smem_addr(sKV), kBoxBytes, 1024);
-      constexpr uint64_t kStageStep = static_cast<uint64_t>(kTile >> 4);
+      const uint32_t k_desc0 = smem_desc_sw128_lo(smem_addr(sKV), 16);
+      const uint32_t v_desc0 = smem_desc_sw128_lo(smem_addr(sKV), kBoxBytes);
+      constexpr uint32_t kStageStep = static_cast<uint32_t>(kTile >> 4);
       // Loads this CTA will consume: a stage is released only if it will be
       // refilled, so that no arrival is left pending when the CTA exits.
       int total_loads = 0;
       for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work;
            idx = next_item(p.work, p.n_work, idx + stride, stride))
         total_loads += 2 * load_item(p, idx).n_kv;
-      int g = 0;        // tile loads consumed so far
-      int k = 0;        // items done
-      uint32_t np[2] = {0, 0};  // P phases consumed per sub-tile
+      int g = 0;                 // tile loads consumed so far
+      int k = 0;                 // current item's index among this CTA's items
+      uint32_t np[2] = {0, 0};   // P phases consumed per sub-tile
+      uint32_t nused[2] = {0, 0};  // items whose O_t went to the epilogue
       bool ok = true;
-      int nidx;
-      for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
-           idx = nidx, ++k) {
-        const ItemInfo it = load_item(p, idx);
-        nidx = next_item(p.work, p.n_work, idx + stride, stride);
-        const bool has_next = nidx < p.n_work;
-        const int n = it.n_kv;
-        const int nt = it.b_valid ? 2 : 1;
-        if (!wait_bar(&ctl.q_full, k & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after_sync();
-        // S_t(0) for both sub-tiles.
+      int idx = next_item(p.work, p.n_work, blockIdx.x, stride);
+      if (idx < p.n_work) {
+        ItemInfo it = load_item(p, idx);
+        int nidx = next_item(p.work, p.n_work, idx + stride, stride);
+        // S_t(0) of the first item.
         {
           const int st = g % NS;
-          if (!wait_bar(&ctl.kv_full[st], (g / NS) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after_sync();
-          for (int t = 0; t < nt; ++t) {
-            issue_qk<D>(tmem + col_s(t), q_desc[t], k_desc0 + st * kStageStep);
-            mma_commit(&ctl.s_full[t]);
-          }
-          if (n == 1 && has_next) mma_commit(&ctl.q_empty);
-          if (g + NS < total_loads) mma_commit(&ctl.kv_empty[st]);
-          ++g;
-        }
-        for (int j = 0; j < n && ok; ++j) {
-          const int gv = g;      // V_j
-          const int gk = g + 1;  // K_{j+1}
-          const bool more = j + 1 < n;
-          const int sv = gv % NS, sk = gk % NS;
-          if (!wait_bar(&ctl.kv_full[sv], (gv / NS) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after_sync();
-          for (int t = 0; t < nt; ++t) {
-            // PV in two halves: the first 64 keys start while the softmax is
-            // still computing the exponentials of the second 64.
-            if (!wait_bar(&ctl.p_half[t][0], np[t] & 1, abort_flag)) { ok = false; break; }
+          ok = wait_bar(&ctl.q_full, 0, abort_flag) &&
+               wait_bar(&ctl.kv_full[st], (g / NS) & 1, abort_flag);
+          if (ok) {
             tc_fence_after_sync();
-            issue_pv<D, 0, 4>(tmem + col_o(t), tmem + col_s(t), v_desc0 + sv * kStageStep, j > 0);
-            if (!wait_bar(&ctl.p_half[t][1], np[t] & 1, abort_flag)) { ok = false; break; }
-            ++np[t];
-            tc_fence_after_sync();
-            issue_pv<D, 4, 8>(tmem + col_o(t), tmem + col_s(t), v_desc0 + sv * kStageStep, true);
-            if (!more) mma_commit(&ctl.o_ready[t]);
-            if (more) {
-              if (t == 0) {
-                // K_{j+1} is needed only now, after PV_a(j) has been queued.
-                if (!wait_bar(&ctl.kv_full[sk], (gk / NS) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after_sync();
-              }
-              issue_qk<D>(tmem + col_s(t), q_desc[t], k_desc0 + sk * kStageStep);
+            for (int t = 0; t < (it.b_valid ? 2 : 1); ++t) {
+              issue_qk<D>(tmem + col_s(t), q_desc[t], k_desc0 + st * kStageStep);
               mma_commit(&ctl.s_full[t]);
             }
+            if (it.n_kv == 1 && nidx < p.n_work) mma_commit(&ctl.q_empty);
+            if (g + NS < total_loads) mma_commit(&ctl.kv_empty[st]);
+            ++g;
           }
-          if (!ok) break;
-          if (gv + NS < total_loads) mma_commit(&ctl.kv_empty[sv]);
-          g = gv + 1;
-          if (more) {
-            if (j + 1 == n - 1 && has_next) mma_commit(&ctl.q_empty);
-            if (gk + NS < total_loads) mma_commit(&ctl.kv_empty[sk]);
-            g = gk + 1;
+        }
+        // One stream of steps across items: step j issues PV_t(j) and the
+        // S_t of the following step, which after an item's last step is the
+        // next item's step 0.
+        while (ok) {
+          const bool has_next = nidx < p.n_work;
+          const ItemInfo nx = has_next ? load_item(p, nidx) : it;
+          for (int j = 0; j < it.n_kv && ok; ++j) {
+            const bool last = j + 1 == it.n_kv;
+            const bool s_next = !last || has_next;  // an S follows this step
+            // the item that S belongs to: its sub-tile b, its last step
+            const bool s_b = last ? nx.b_valid : it.b_valid;
+            const bool s_is_last = last ? nx.n_kv == 1 : j + 2 == it.n_kv;
+            const int gv = g;      // V_j
+            const int gk = g + 1;  // the following K
+            const int sv = gv % NS, sk = gk % NS;
+            if (!wait_bar(&ctl.kv_full[sv], (gv / NS) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after_sync();
+            bool k_ready = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (t == 0 || it.b_valid) {
+                if (j == 0 && nused[t] > 0) {
+                  // O_t still holds the previous item's output: the first
+                  // PV_t overwrites it only once the epilogue has drained it.
+                  if (!wait_bar(&ctl.o_free[t], (nused[t] - 1) & 1, abort_flag)) { ok = false; break; }
+                }
+                // PV in two halves: the first 64 keys start while the softmax
+                // is still computing the exponentials of the second 64.
+                if (!wait_bar(&ctl.p_half[t][0], np[t] & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after_sync();
+                issue_pv<D, 0, 4>(tmem + col_o(t), tmem + col_s(t), v_desc0 + sv * kStageStep, j > 0);
+                if (!wait_bar(&ctl.p_half[t][1], np[t] & 1, abort_flag)) { ok = false; break; }
+                ++np[t];
+                tc_fence_after_sync();
+                issue_pv<D, 4, 8>(tmem + col_o(t), tmem + col_s(t), v_desc0 + sv * kStageStep, true);
+                if (last) {
+                  mma_commit(&ctl.o_ready[t]);
+                  ++nused[t];
+                }
+              }
+              if (s_next && (t == 0 || s_b)) {
+                if (!k_ready) {
+                  // The following K is needed only now, after PV_a(j) has
+                  // been queued; a new item's first S also needs its Q.
+                  if (!wait_bar(&ctl.kv_full[sk], (gk / NS) & 1, abort_flag)) { ok = false; break; }
+                  if (last && !wait_bar(&ctl.q_full, (k + 1) & 1, abort_flag)) { ok = false; break; }
+                  tc_fence_after_sync();
+                  k_ready = true;
+                }
+                issue_qk<D>(tmem + col_s(t), q_desc[t], k_desc0 + sk * kStageStep);
+                mma_commit(&ctl.s_full[t]);
+              }
+            }
+            if (!ok) break;
+            if (gv + NS < total_loads) mma_commit(&ctl.kv_empty[sv]);
+            g = gv + 1;
+            if (s_next) {
+              // Q is free once the last S of its item has been issued (the
+              // producer then loads the next item's Q over it).
+              const bool after = last ? (nidx < p.n_work &&
+                                         next_item(p.work, p.n_work, nidx + stride, stride) < p.n_work)
+                                      : has_next;
+              if (s_is_last && after) mma_commit(&ctl.q_empty);
+              if (gk + NS < total_loads) mma_commit(&ctl.kv_empty[sk]);
+              g = gk + 1;
+            }
           }
+          if (!ok || !has_next) break;
+          it = nx;
+          idx = nidx;
+          nidx = next_item(p.work, p.n_work, idx + stride, stride);
+          ++k;
         }
       }
       if (!ok) {
@@ -425,6 +485,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         wait_slow(&ctl.drain, 0, nullptr, kDrainLimitNs);
       }
     }
+  }
   } else if (warp < 8) {
     // ----------------------------------------------------------- softmax ---
     setmaxnreg_inc<kSoftmaxRegs>();
@@ -437,7 +498,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f32x2(sl2, sl2);
     uint32_t ns = 0;  // S phases consumed
-    uint32_t no = 0;  // O phases consumed
     bool ok = true;
     for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
          idx = next_item(p.work, p.n_work, idx + stride, stride)) {
@@ -457,7 +517,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float s[128];
         {
           uint32_t sr[128];
-          tmem_ld128_sync(s_tmem, sr);
+          tmem_ld64x2_sync(s_tmem, sr);
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
         }
@@ -522,12 +582,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l += (la0 + la1) + (lb0 + lb1);
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16 rows of this sub-tile ----
-      if (!warp_wait_bar(&ctl.o_ready[t], no & 1, abort_flag)) { ok = false; break; }
-      ++no;
-      tc_fence_after_sync();
+      // ---- end of the item: the row's log-normaliser, and 1/l for the
+      // epilogue warps, which drain O_t while this warp starts the next item.
       const int q_row = it.q0 + t * kSubM + row;
-      const float inv_l = 1.0f / l;
       // log of the row's softmax normaliser, sum_u exp(s_u * scale), for the
       // backward pass: m and l are in the exp2 domain of s * scale * log2(e).
       if (p.lse && row_in) {
@@ -535,44 +592,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (in_bounds(li, static_cast<long long>(p.heads) * p.total_tokens))
           p.lse[li] = (m + log2f(l)) * 0.6931471805599453f;
       }
-      // O / l in 64-dim halves through this warp's 4 KB of shared memory:
-      // each lane writes its row (128 bytes, 16-byte chunk c at c ^ (row % 8)),
-      // then each store instruction of the warp writes four whole 128-byte row
-      // segments (eight lanes per row) instead of 32 scattered 16-byte pieces.
-      uint8_t* stage = sOut + warp * 4096;
-      const int rr0 = lane >> 3;  // first row this lane stores, then every 4th
-      const int cc = lane & 7;    // 16-byte chunk of the row this lane stores
-      const int row0 = it.q0 + t * kSubM + wl * 32;  // token of the warp's first row
+      ctl.inv_l[t][row] = 1.0f / l;
+      mbar_arrive(&ctl.stat_ready[t]);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue ---
+    setmaxnreg_dec<kEpilogueRegs>();
+    const int wq = warp % 4;  // TMEM lane quarter: rows 32 * wq .. of each sub-tile
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    uint8_t* stage = sOut + (warp - kEpilogueWarp0) * 4096;
+    const int rr0 = lane >> 3;  // first row this lane stores, then every 4th
+    const int cc = lane & 7;    // 16-byte chunk of the row this lane stores
+    uint32_t no[2] = {0, 0};    // items drained per sub-tile
+    bool ok = true;
+    for (int idx = next_item(p.work, p.n_work, blockIdx.x, stride); idx < p.n_work && ok;
+         idx = next_item(p.work, p.n_work, idx + stride, stride)) {
+      const ItemInfo it = load_item(p, idx);
       const int row_end = it.seg_start + it.seg_len;
+      for (int t = 0; t < (it.b_valid ? 2 : 1); ++t) {
+        if (!warp_wait_bar(&ctl.stat_ready[t], no[t] & 1, abort_flag) ||
+            !warp_wait_bar(&ctl.o_ready[t], no[t] & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ++no[t];
+        tc_fence_after_sync();
+        const float inv_l = ctl.inv_l[t][row];
+        const uint32_t o_tmem = tmem + lane_off + col_o(t);
+        const int row0 = it.q0 + t * kSubM + wq * 32;  // token of the warp's first row
+        // O / l in 64-dim halves through this warp's 4 KB of shared memory:
+        // each lane writes its row (128 bytes, 16-byte chunk c at c ^ (row % 8)),
+        // then each store instruction of the warp writes four whole 128-byte
+        // row segments (eight lanes per row) instead of 32 scattered 16-byte
+        // pieces.
 #pragma unroll 1
-      for (int half = 0; half < D / 64; ++half) {
+        for (int half = 0; half < D / 64; ++half) {
 #pragma unroll
-        for (int c32 = 0; c32 < 2; ++c32) {
-          uint32_t r[32];
-          tmem_ld32_sync(o_tmem + 64 * half + 32 * c32, r);
+          for (int c16 = 0; c16 < 4; ++c16) {
+            uint32_t r[16];
+            tmem_ld16_sync(o_tmem + 64 * half + 16 * c16, r);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(r[8 * v4 + 0]) * inv_l, __uint_as_float(r[8 * v4 + 1]) * inv_l);
-            o.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * inv_l, __uint_as_float(r[8 * v4 + 3]) * inv_l);
-            o.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * inv_l, __uint_as_float(r[8 * v4 + 5]) * inv_l);
-            o.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * inv_l, __uint_as_float(r[8 * v4 + 7]) * inv_l);
-            const int c = 4 * c32 + v4;
-            *reinterpret_cast<uint4*>(stage + lane * 128 + ((c ^ (lane & 7)) << 4)) = o;
+            for (int v4 = 0; v4 < 2; ++v4) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v4 + 0]) * inv_l, __uint_as_float(r[8 * v4 + 1]) * inv_l);
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * inv_l, __uint_as_float(r[8 * v4 + 3]) * inv_l);
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * inv_l, __uint_as_float(r[8 * v4 + 5]) * inv_l);
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * inv_l, __uint_as_float(r[8 * v4 + 7]) * inv_l);
+              const int c = 2 * c16 + v4;
+              *reinterpret_cast<uint4*>(stage + lane * 128 + ((c ^ (lane & 7)) << 4)) = o;
+            }
           }
+          if (half == D / 64 - 1) {
+            // O_t has been read: the next item's first PV_t may overwrite it.
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl.o_free[t]);
+          }
+          __syncwarp();
+#pragma unroll 2
+          for (int i = 0; i < 8; ++i) {
+            const int rr = 4 * i + rr0;
+            const uint4 o = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((cc ^ (rr & 7)) << 4));
+            const int tok = row0 + rr;
+            const size_t oi = (static_cast<size_t>(tok) * p.heads + it.head) * (D / 8) + 8 * half + cc;
+            if (tok < row_end &&
+                in_bounds(oi, static_cast<long long>(p.total_tokens) * p.heads * (D / 8)))
+              reinterpret_cast<uint4*>(p.out)[oi] = o;
+          }
+          __syncwarp();
         }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + rr0;
-          const uint4 o = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((cc ^ (rr & 7)) << 4));
-          const int tok = row0 + rr;
-          const size_t oi = (static_cast<size_t>(tok) * p.heads + it.head) * (D / 8) + 8 * half + cc;
-          if (tok < row_end &&
-              in_bounds(oi, static_cast<long long>(p.total_tokens) * p.heads * (D / 8)))
-            reinterpret_cast<uint4*>(p.out)[oi] = o;
-        }
-        __syncwarp();
       }
     }
   }

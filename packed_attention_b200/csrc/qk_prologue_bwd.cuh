@@ -55,52 +55,21 @@ __global__ void __launch_bounds__(kPrologueThreads) bwd_delta_kernel(
   }
 }
 
-// The (cos, sin) of the 4 pairs a thread owns, for token t (text: identity).
-// Same positions and angle formation as the forward prologue.
+// The (cos, sin) of the 4 pairs a thread owns, for token t (text: identity),
+// from the forward prologue's positions and angles; returns whether t is text.
 template <int D>
 __device__ __forceinline__ bool token_rotation(const int32_t* __restrict__ cu_seqlens,
                                                const mf_segment* __restrict__ segs, int n_samples,
                                                int t, int e0, int frame_dims, float (&cs)[4],
                                                float (&sn)[4]) {
-  int lo = 0, hi = n_samples;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(cu_seqlens + mid) <= t) lo = mid; else hi = mid;
-  }
-  const int start = __ldg(&segs[lo].start);
-  const int n_text = __ldg(&segs[lo].n_text);
-  const int gw = __ldg(&segs[lo].grid_w);
-  const int hw = __ldg(&segs[lo].grid_h) * gw;
-  const int j = t - start;
-  if (j < n_text) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) { cs[i] = 1.0f; sn[i] = 0.0f; }
-    return true;
-  }
-  const int spatial = (D - frame_dims) / 2;
-  const int frame = (j - n_text) / hw;
-  const int p = (j - n_text) % hw;
-  const int row = p / gw, col = p % gw;
-  constexpr double kLog2Base = 13.287712379549449;
-  constexpr double kTwoPi = 6.283185307179586;
-  constexpr double kInvTwoPi = 0.15915494309189535;
+  const TokenPos tp = token_position(cu_seqlens, segs, n_samples, t);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int e = e0 + 2 * i;
-    int pos, first, width;
-    if (e < frame_dims) {
-      pos = frame; first = 0; width = frame_dims;
-    } else if (e < frame_dims + spatial) {
-      pos = row; first = frame_dims; width = spatial;
-    } else {
-      pos = col; first = frame_dims + spatial; width = spatial;
-    }
-    const double theta = exp2(-(2.0 * ((e - first) / 2) / width) * kLog2Base);
-    double ang = static_cast<double>(pos) * theta;
-    ang -= kTwoPi * rint(ang * kInvTwoPi);
-    sincosf(static_cast<float>(ang), &sn[i], &cs[i]);
+    const float2 r = pair_cos_sin<D>(tp, e0 / 2 + i, frame_dims);
+    cs[i] = r.x;
+    sn[i] = r.y;
   }
-  return false;
+  return tp.text;
 }
 
 // dq, dk (bf16) from dq_hat, dk_hat (fp32) and the raw q, k; partial gamma
