@@ -127,45 +127,6 @@ bool prepare_attention_kernel() {
   return ok[dev];
 }
 
-// The prologue's chunking: a chunk of tps tokens holds at least ~8 KB of q
-// and k rows (tps <= 16), and the ring takes as many chunks as fit the
-// shared-memory budget next to the compute warps' tables (at most
-// kProMaxStages). False if not even two fit (heads * head_dim above ~24,000).
-bool prologue_plan(int heads, int head_dim, mf::ProloguePlan* pp, size_t* smem) {
-  const size_t tok_bytes = static_cast<size_t>(heads) * head_dim * 2;
-  size_t tps = 8192 / (2 * tok_bytes);
-  tps = tps < 1 ? 1 : (tps > static_cast<size_t>(mf::kProMaxTps) ? mf::kProMaxTps : tps);
-  const size_t stage = mf::prologue_stage_bytes(static_cast<int>(tps), heads, head_dim);
-  const size_t tables = (mf::kProComputeThreads / 32) *
-                        mf::prologue_table_bytes(static_cast<int>(tps), head_dim);
-  size_t stages = (mf::kProSmemBudget - tables) / stage;
-  if (stages > static_cast<size_t>(mf::kProMaxStages)) stages = mf::kProMaxStages;
-  if (stages < 2) return false;
-  // Two stages per compute warp when they fit, else one; with fewer than 8
-  // stages, one warp per stage.
-  const size_t warps = stages >= 8 ? 8 : stages;
-  stages = stages / warps * warps;
-  pp->tps = static_cast<int>(tps);
-  pp->stages = static_cast<int>(stages);
-  pp->warps = static_cast<int>(warps);
-  *smem = mf::prologue_smem_bytes(*pp, heads, head_dim);
-  return true;
-}
-
-template <int D>
-bool prepare_prologue_kernel() {
-  static std::once_flag once[kMaxDevices];
-  static bool ok[kMaxDevices];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  std::call_once(once[dev], [dev] {
-    ok[dev] = cudaFuncSetAttribute(mf::qk_prologue_kernel<D>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   mf::kProSmemBudget) == cudaSuccess;
-  });
-  return ok[dev];
-}
-
 // Dynamic shared memory of the two backward attention kernels, set once per device.
 template <int D>
 bool prepare_bwd_kernels() {
@@ -238,24 +199,17 @@ extern "C" mf_status mf_qk_prologue_3d(const void* q, const void* k, const float
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  mf::ProloguePlan pp;
-  size_t smem = 0;
-  if (!prologue_plan(heads, head_dim, &pp, &smem)) return MF_ERR_UNSUPPORTED;
-  const int sms = sm_count();
-  if (sms <= 0) return MF_ERR_CUDA;
-  const int n_chunks = (total_tokens + pp.tps - 1) / pp.tps;
-  const unsigned grid = static_cast<unsigned>(n_chunks < sms ? n_chunks : sms);
+  const int tok_per_block = mf::kPrologueThreads / (head_dim / 8);
+  const unsigned grid = static_cast<unsigned>((total_tokens + tok_per_block - 1) / tok_per_block);
   if (head_dim == 128) {
-    if (!prepare_prologue_kernel<128>()) return MF_ERR_CUDA;
-    mf::qk_prologue_kernel<128><<<grid, mf::kProThreads, smem, s>>>(
+    mf::qk_prologue_kernel<128><<<grid, mf::kPrologueThreads, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
-        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims, pp,
+        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims,
         reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat));
   } else {
-    if (!prepare_prologue_kernel<64>()) return MF_ERR_CUDA;
-    mf::qk_prologue_kernel<64><<<grid, mf::kProThreads, smem, s>>>(
+    mf::qk_prologue_kernel<64><<<grid, mf::kPrologueThreads, 0, s>>>(
         static_cast<const uint4*>(q), static_cast<const uint4*>(k), g_q_text, g_q_img, g_k_text,
-        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims, pp,
+        g_k_img, cu_seqlens_dev, segs_dev, n_samples, total_tokens, heads, eps, frame_dims,
         reinterpret_cast<uint4*>(ws + w.q_hat), reinterpret_cast<uint4*>(ws + w.k_hat));
   }
   return cudaGetLastError() == cudaSuccess ? MF_OK : MF_ERR_CUDA;

@@ -19,25 +19,13 @@
 // F = 0 is the 2D rotation above.
 //
 // HBM-bound: it reads q and k and writes q_hat and k_hat once (8 * T * H * d
-// bytes), a copy-shaped stream. Persistent: one CTA per SM takes a
-// contiguous range of chunks of `tps` tokens (every head of a token is one
-// contiguous H*d*2-byte row of q and of k).
-//   warp 8 (1 lane)  producer: bulk-copies each chunk's q and k rows into a
-//                    ring of shared-memory stages (one mbarrier per stage,
-//                    completion counted in bytes), so that many chunks are
-//                    in flight however long the math takes.
-//   warps 0-7        each on its own chunks (warp w of W: the CTA's chunks
-//                    w, w + W, ..., in stages of its own): first the (cos, sin) of every rotation
-//                    pair of the chunk's tokens into the warp's small shared
-//                    table (one sincos per pair and token, not per head),
-//                    then each (token, head) row of q and k: d/8 lanes per
-//                    row, 8 consecutive dims (one 16-byte vector) each, the
-//                    mean square by shuffles within the row's lanes; 16-byte
-//                    stores of q_hat, k_hat that cover whole 512-byte row
-//                    pairs per warp.
-// Every wait is bounded; a wait that runs out records MF_ERR_TIMEOUT, every
-// warp leaves its loop, and the producer waits (bounded) for its copies in
-// flight.
+// bytes). Layout of the work: a group of d/8 threads owns one token and
+// loops over its heads; each thread holds 8 consecutive dims (one 16-byte vector) of q and of k, so a warp
+// reads and writes whole 256-byte rows, and it requests the next head's
+// vectors before it works on the current one. The token's position, gammas
+// and the 4 (cos, sin) pairs a thread needs are computed once per token
+// (theta of each pair once per block) and reused for all heads and for both
+// q and k.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -53,11 +41,6 @@ namespace mf {
 // Threads per block of the backward's per-token kernels (delta, norm backward).
 constexpr int kPrologueThreads = 256;
 
-constexpr int kProComputeThreads = 256;  // warps 0-7
-constexpr int kProThreads = kProComputeThreads + 32;
-constexpr int kProMaxStages = 16;
-constexpr int kProMaxTps = 16;
-constexpr int kProSmemBudget = 200 * 1024;  // stages + tables, below the 227 KB per CTA
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -152,188 +135,113 @@ __device__ __forceinline__ float2 pair_cos_sin(const TokenPos& tp, int pair, int
   return rotation_cos_sin(pos, pair_theta(e_in, width));
 }
 
-// Chunking and staging of one launch, chosen on the host.
-struct ProloguePlan {
-  int tps;     // tokens per chunk
-  int stages;  // ring depth, a multiple of warps
-  int warps;   // compute warps in use (<= 8); warp w owns stages w, w + warps, ...
-};
-
-__host__ __device__ constexpr size_t prologue_stage_bytes(int tps, int heads, int d) {
-  return 2 * static_cast<size_t>(tps) * heads * d * 2;  // q rows, then k rows
-}
-
-// Per compute warp: the (cos, sin) of every pair of its chunk's tokens, then
-// their text flags.
-__host__ __device__ constexpr size_t prologue_table_bytes(int tps, int d) {
-  return static_cast<size_t>(tps) * (d / 2) * 8 + kProMaxTps * 4;
-}
-
-__host__ __device__ constexpr size_t prologue_smem_bytes(ProloguePlan pp, int heads, int d) {
-  return pp.stages * prologue_stage_bytes(pp.tps, heads, d) +
-         (kProComputeThreads / 32) * prologue_table_bytes(pp.tps, d);
-}
-
 template <int D>
-__global__ void __launch_bounds__(kProThreads, 1) qk_prologue_kernel(
+__global__ void __launch_bounds__(kPrologueThreads, 4) qk_prologue_kernel(
     const uint4* __restrict__ q, const uint4* __restrict__ k, const float* __restrict__ gq_text,
     const float* __restrict__ gq_img, const float* __restrict__ gk_text,
     const float* __restrict__ gk_img, const int32_t* __restrict__ cu_seqlens,
     const mf_segment* __restrict__ segs, int n_samples, int total_tokens, int heads, float eps,
-    int frame_dims, ProloguePlan plan, uint4* __restrict__ q_hat, uint4* __restrict__ k_hat) {
-  constexpr int kTpr = D / 8;              // threads (16-byte vectors) per row
-  constexpr int kRowsPerPass = 32 / kTpr;  // rows a warp handles at once
-  constexpr int kWarps = kProComputeThreads / 32;
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint64_t full[kProMaxStages], empty[kProMaxStages];
+    int frame_dims, uint4* __restrict__ q_hat, uint4* __restrict__ k_hat) {
+  constexpr int kVecPerRow = D / 8;  // 16-byte vectors per row
+  constexpr int kTokPerBlock = kPrologueThreads / kVecPerRow;
   __shared__ double s_theta[D / 2];
   __shared__ int32_t s_axis[D / 2];
-  __shared__ int32_t abort_word;
-  volatile int32_t* abort_flag = &abort_word;
 
-  const int tps = plan.tps, S = plan.stages, W = plan.warps;
-  const size_t tok_bytes = static_cast<size_t>(heads) * D * 2;
-  const size_t stage_bytes = prologue_stage_bytes(tps, heads, D);
+  const int vec = threadIdx.x % kVecPerRow;
+  const int t_raw = blockIdx.x * kTokPerBlock + threadIdx.x / kVecPerRow;
+  // Threads past the last token compute on a valid token (so every lane of
+  // the warp takes part in the shuffles) and store nothing.
+  const bool active = t_raw < total_tokens;
+  const int t = active ? t_raw : total_tokens - 1;
+  const size_t row0 = static_cast<size_t>(t) * heads * kVecPerRow + vec;
+  const long long n_vec = static_cast<long long>(total_tokens) * heads * kVecPerRow;
 
-  const int n_chunks = (total_tokens + tps - 1) / tps;
-  const int c0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_chunks / gridDim.x);
-  const int c1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_chunks / gridDim.x);
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    abort_word = 0;
-    fence_mbarrier_init();
+  // The first head's q and k are requested before any setup.
+  uint4 qv = make_uint4(0, 0, 0, 0), kv = make_uint4(0, 0, 0, 0);
+  if (in_bounds(row0, n_vec)) {
+    qv = __ldg(q + row0);
+    kv = __ldg(k + row0);
   }
-  // theta and axis of every pair, once per CTA
-  for (int pr = threadIdx.x; pr < D / 2; pr += blockDim.x) {
+  // theta and axis of every pair, once per block
+  for (int pr = threadIdx.x; pr < D / 2; pr += kPrologueThreads) {
     int e_in, width;
     s_axis[pr] = pair_axis(pr, D, frame_dims, e_in, width);
     s_theta[pr] = pair_theta(e_in, width);
   }
   __syncthreads();
 
-  if (warp == kWarps) {
-    // ---------------------------------------------------------- producer ---
-    if (lane == 0) {
-      const size_t tensor_bytes = static_cast<size_t>(total_tokens) * tok_bytes;
-      int i = 0;
-      bool ok = true;
-      for (int c = c0; c < c1; ++c, ++i) {
-        const int s = i % S;
-        if (i >= S && !wait_bar(&empty[s], ((i / S) - 1) & 1, abort_flag)) { ok = false; break; }
-        const int t0 = c * tps;
-        const int ntok = min(tps, total_tokens - t0);
-        const uint32_t bytes = static_cast<uint32_t>(ntok * tok_bytes);
-        const uint8_t* src_q = reinterpret_cast<const uint8_t*>(q) + t0 * tok_bytes;
-        const uint8_t* src_k = reinterpret_cast<const uint8_t*>(k) + t0 * tok_bytes;
-        if (!in_span(src_q, bytes, q, tensor_bytes) || !in_span(src_k, bytes, k, tensor_bytes)) {
-          ok = false;
-          *abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[s], 2 * bytes);
-        bulk_load(smem + s * stage_bytes, src_q, bytes, &full[s]);
-        bulk_load(smem + s * stage_bytes + tps * tok_bytes, src_k, bytes, &full[s]);
-      }
-      if (!ok) {
-        // Every copy already issued must land before the CTA exits: wait for
-        // the stages of the last min(i, S) chunks (earlier ones were consumed).
-        for (int j = i - S > 0 ? i - S : 0; j < i; ++j)
-          wait_slow(&full[j % S], (j / S) & 1, nullptr, kDrainLimitNs);
-      }
+  // The token's position, gammas and the (cos, sin) of the 4 pairs this
+  // thread owns: once per token, for all its heads and for both q and k.
+  const TokenPos tp = token_position(cu_seqlens, segs, n_samples, t);
+  const int e0 = vec * 8;  // first dim this thread owns
+  float cs[4], sn[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int pair = e0 / 2 + i;
+    float2 r = make_float2(1.0f, 0.0f);
+    if (!tp.text) {
+      const int axis = s_axis[pair];
+      r = rotation_cos_sin(axis == 0 ? tp.frame : (axis == 1 ? tp.row : tp.col), s_theta[pair]);
     }
-    return;
+    cs[i] = r.x;
+    sn[i] = r.y;
+  }
+  float gq[8], gk[8];
+  {
+    const float* gqs = tp.text ? gq_text : gq_img;
+    const float* gks = tp.text ? gk_text : gk_img;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      gq[i] = __ldg(gqs + e0 + i);
+      gk[i] = __ldg(gks + e0 + i);
+    }
   }
 
-  // ------------------------------------------------------------- compute ---
-  // Warp w takes this CTA's chunks w, w + W, w + 2W, ... on its own: the
-  // rotation table of its chunk, then the chunk's 2 * tokens * heads rows.
-  // Chunk i sits in stage i % S and S is a multiple of W, so a stage only
-  // ever holds one warp's chunks, in that warp's order: each parity wait is
-  // on the phase right after the one the warp consumed last.
-  if (warp >= W) return;
-  const int vec = lane % kTpr;
-  const int e0 = vec * 8;  // first dim this thread owns
-  float g[4][8];           // q_text, q_img, k_text, k_img: this thread's 8 dims
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    g[0][m] = __ldg(gq_text + e0 + m);
-    g[1][m] = __ldg(gq_img + e0 + m);
-    g[2][m] = __ldg(gk_text + e0 + m);
-    g[3][m] = __ldg(gk_img + e0 + m);
-  }
-  float2* table = reinterpret_cast<float2*>(smem + S * stage_bytes +
-                                            warp * prologue_table_bytes(tps, D));
-  int32_t* text = reinterpret_cast<int32_t*>(table + tps * (D / 2));
   const float inv_d = 1.0f / D;
-  const long long n_vec = static_cast<long long>(total_tokens) * heads * kTpr;
-  for (int i = warp; c0 + i < c1; i += W) {
-    const int s = i % S;
-    if (!warp_wait_bar(&full[s], (i / S) & 1, abort_flag)) break;
-    const int t0 = (c0 + i) * tps;
-    const int ntok = min(tps, total_tokens - t0);
-    // (cos, sin) of every pair of every token of the chunk, and its modality.
-    for (int pr = lane; pr < ntok * (D / 2); pr += 32) {
-      const int tl = pr / (D / 2), pair = pr % (D / 2);
-      const TokenPos tp = token_position(cu_seqlens, segs, n_samples, t0 + tl);
-      if (tp.text) {
-        table[pr] = make_float2(1.0f, 0.0f);
-      } else {
-        const int axis = s_axis[pair];
-        table[pr] = rotation_cos_sin(axis == 0 ? tp.frame : (axis == 1 ? tp.row : tp.col),
-                                     s_theta[pair]);
+#pragma unroll 2
+  for (int h = 0; h < heads; ++h) {
+    const size_t idx = row0 + static_cast<size_t>(h) * kVecPerRow;
+    // the next head's loads go out before this head's math
+    uint4 qn = make_uint4(0, 0, 0, 0), kn = make_uint4(0, 0, 0, 0);
+    if (h + 1 < heads) {
+      const size_t nidx = idx + kVecPerRow;
+      if (in_bounds(nidx, n_vec)) {
+        qn = __ldg(q + nidx);
+        kn = __ldg(k + nidx);
       }
-      if (pair == 0) text[tl] = tp.text ? 1 : 0;
     }
-    __syncwarp();
-    const uint8_t* stage = smem + s * stage_bytes;
-    const int rows = 2 * ntok * heads;  // q rows of the chunk, then its k rows
-    const int rows_q = ntok * heads;
-#pragma unroll 4
-    for (int r0 = 0; r0 < rows; r0 += kRowsPerPass) {
-      const int r = r0 + lane / kTpr;
-      const bool valid = r < rows;
-      // A row past the chunk's end computes on its last row (so that every
-      // thread of the row group takes part in the shuffles) and stores nothing.
-      const int re = valid ? r : rows - 1;
-      const int kk = re >= rows_q;      // 0: q, 1: k
-      const int rr = re - kk * rows_q;  // (token, head) row within the chunk
-      const int tl = rr / heads;
-      float x[8];
-      unpack8(*reinterpret_cast<const uint4*>(stage + kk * tps * tok_bytes +
-                                              static_cast<size_t>(rr) * D * 2 + vec * 16),
-              x);
-      float ss = 0.f;
+    float xq[8], xk[8];
+    unpack8(qv, xq);
+    unpack8(kv, xk);
+    float ssq = 0.f, ssk = 0.f;
 #pragma unroll
-      for (int m = 0; m < 8; ++m) ss = fmaf(x[m], x[m], ss);
-#pragma unroll
-      for (int o = kTpr / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, kTpr);
-      const float rn = rsqrtf(fmaf(ss, inv_d, eps));
-      const bool tx = text[tl] != 0;
-      float gm[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) gm[m] = kk ? (tx ? g[2][m] : g[3][m]) : (tx ? g[0][m] : g[1][m]);
-      const float4 cs01 = *reinterpret_cast<const float4*>(table + tl * (D / 2) + 4 * vec);
-      const float4 cs23 = *reinterpret_cast<const float4*>(table + tl * (D / 2) + 4 * vec + 2);
-      const float cs[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
-      const float sn[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
-      float y[8];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float a = x[2 * m] * rn * gm[2 * m], b = x[2 * m + 1] * rn * gm[2 * m + 1];
-        y[2 * m] = a * cs[m] - b * sn[m];
-        y[2 * m + 1] = a * sn[m] + b * cs[m];
-      }
-      const size_t idx = (static_cast<size_t>(t0) * heads + rr) * kTpr + vec;
-      if (valid && in_bounds(idx, n_vec)) (kk ? k_hat : q_hat)[idx] = pack8(y);
+    for (int i = 0; i < 8; ++i) {
+      ssq = fmaf(xq[i], xq[i], ssq);
+      ssk = fmaf(xk[i], xk[i], ssk);
     }
-    // This warp is done with the stage and its table.
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+    for (int o = kVecPerRow / 2; o > 0; o >>= 1) {
+      ssq += __shfl_xor_sync(0xffffffffu, ssq, o, kVecPerRow);
+      ssk += __shfl_xor_sync(0xffffffffu, ssk, o, kVecPerRow);
+    }
+    const float rq = rsqrtf(fmaf(ssq, inv_d, eps));
+    const float rk = rsqrtf(fmaf(ssk, inv_d, eps));
+    float yq[8], yk[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float qa = xq[2 * i] * rq * gq[2 * i], qb = xq[2 * i + 1] * rq * gq[2 * i + 1];
+      const float ka = xk[2 * i] * rk * gk[2 * i], kb = xk[2 * i + 1] * rk * gk[2 * i + 1];
+      yq[2 * i] = qa * cs[i] - qb * sn[i];
+      yq[2 * i + 1] = qa * sn[i] + qb * cs[i];
+      yk[2 * i] = ka * cs[i] - kb * sn[i];
+      yk[2 * i + 1] = ka * sn[i] + kb * cs[i];
+    }
+    if (active && in_bounds(idx, n_vec)) {
+      q_hat[idx] = pack8(yq);
+      k_hat[idx] = pack8(yk);
+    }
+    qv = qn;
+    kv = kn;
   }
 }
 
