@@ -17,7 +17,8 @@ import torch
 import oracle
 import packed_attention_b200 as pa
 from packed_attention_b200.workloads import CFG_PACKS, Workload, make_inputs, random_pack
-from test_gpu_parity import MAX_ABS, REL_RMS, bf16_to_f64, errors, run_gpu, sample_rows
+from test_gpu_parity import (MAX_ABS, REL_RMS, bf16_to_f64, compare_every_element, errors,
+                             run_gpu, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,14 +50,11 @@ def test_cfg_pack_equals_separate_branches(cuda_device, name):
 
 @pytest.mark.parametrize("name", sorted(CFG_PACKS))
 def test_cfg_pack_matches_oracle(cuda_device, name):
+    """The packed CFG forward against the oracle on every element."""
     w = CFG_PACKS[name].packed()
     inp = make_inputs(w)
     _, _, out = run_gpu(w, inp, cuda_device)
-    rows = sample_rows(w, np.random.default_rng(7))
-    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps, rows=rows)
-    got = bf16_to_f64(out).reshape(-1, w.head_dim)[rows]
-    max_abs, rel_rms = errors(got, ref)
-    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
+    compare_every_element(w, inp, out, name)
 
 
 @pytest.mark.parametrize("trial", range(6))

@@ -214,7 +214,8 @@ def oracle_full_output(w: Workload, inp):
     if os.path.exists(path):
         return np.load(path).astype(np.float64), 0.0
     t0 = time.perf_counter()
-    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps)
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps,
+                            frame_dims=w.rope_frame_dims)
     sec = time.perf_counter() - t0
     os.makedirs(CACHE_DIR, exist_ok=True)
     tmp = path + f".tmp{os.getpid()}.npy"
@@ -223,16 +224,12 @@ def oracle_full_output(w: Workload, inp):
     return ref, sec
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
-def test_full_size_config_every_element(cuda_device, cfg):
-    """Every element of the full-size pack's output against the oracle: the
-    bar over all T*H*d elements, and the same bar on each head alone (so that
-    an error confined to some heads cannot hide in the average)."""
-    w = WORKLOADS[cfg]
-    inp = make_inputs(w)
-    _, _, out = run_gpu(w, inp, cuda_device)
+def compare_every_element(w: Workload, inp, out, tag):
+    """Every element of ``out`` (bf16 [T, H, d] on the GPU) against the
+    oracle: the bar over all T*H*d elements, and the same bar on each head
+    alone (so that an error confined to some heads cannot hide in the
+    average)."""
     got = out.float().cpu().numpy()
-    del out
     assert np.all(np.isfinite(got))
     ref, oracle_s = oracle_full_output(w, inp)
     sq_diff = sq_ref = 0.0
@@ -250,7 +247,7 @@ def test_full_size_config_every_element(cuda_device, cfg):
     report = os.environ.get("MF_PARITY_REPORT")
     if report:
         with open(report, "a") as f:
-            f.write(json.dumps({"config": cfg, "workload": w.name, "compared": "every element",
+            f.write(json.dumps({"config": tag, "workload": w.name, "compared": "every element",
                                 "elements": int(got.size), "max_abs": max_abs,
                                 "rel_rms": rel_rms,
                                 "worst_head_rel_rms": max(r for _, r in per_head),
@@ -258,6 +255,15 @@ def test_full_size_config_every_element(cuda_device, cfg):
     assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
     bad = [(h, m, r) for h, (m, r) in enumerate(per_head) if m > MAX_ABS or r > REL_RMS]
     assert not bad, bad
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_full_size_config_every_element(cuda_device, cfg):
+    """Every element of the full-size pack's output against the oracle."""
+    w = WORKLOADS[cfg]
+    inp = make_inputs(w)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    compare_every_element(w, inp, out, cfg)
 
 
 # --------------------------------------------------------------- hygiene ---

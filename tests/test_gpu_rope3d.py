@@ -90,6 +90,16 @@ def test_edit_pack_3d_sampled_rows(cuda_device):
     assert np.sqrt(np.mean((ref - ref2d) ** 2)) > 10 * REL_RMS * np.sqrt(np.mean(ref ** 2))
 
 
+def test_edit_pack_3d_every_element(cuda_device):
+    """The 1024^2 edit pack with the frame axis: every element of the output
+    against the oracle."""
+    from test_gpu_parity import compare_every_element
+    w = EDIT3D
+    inp = make_inputs(w)
+    _, _, out = run3d(w, inp, cuda_device)
+    compare_every_element(w, inp, out, w.name)
+
+
 @pytest.mark.parametrize("trial", range(4))
 def test_random_packs_3d_full_compare(cuda_device, trial):
     rng = np.random.default_rng(800 + trial)
