@@ -597,6 +597,13 @@ def main():
         if e2 is not None:
             e2.record(stream)
 
+    # The clock sampler starts before the warm-up (nvidia-smi needs a moment
+    # to come up), so that the timed region follows the warm-up with no idle
+    # gap in which the clocks could drop.
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -606,12 +613,8 @@ def main():
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local_rank) if rank == 0 else None
     barrier()
     torch.cuda.synchronize()
-    if sampler:
-        sampler.start()
-        time.sleep(0.3)
     start.record(stream)
     for i in range(K):
         step(*evs[i])
@@ -628,8 +631,9 @@ def main():
     step_steps = [e[0].elapsed_time(e[2]) for e in evs]
     pro_ms = sum(pro_steps) / K
     att_ms = sum(att_steps) / K
-    per_step = [statistics.median(step_steps), min(step_steps), statistics.median(pro_steps),
-                min(pro_steps), statistics.median(att_steps), min(att_steps)]
+    per_step = [statistics.median(step_steps), min(step_steps), max(step_steps),
+                statistics.median(pro_steps), min(pro_steps), statistics.median(att_steps),
+                min(att_steps), max(att_steps)]
     total_ms, pro_ms, att_ms, *per_step = max_over_ranks(
         [total_ms, pro_ms, att_ms, *per_step], world, dev)
 
@@ -702,8 +706,9 @@ def main():
         "tokens_per_s": tokens_per_s,
         "pct_of_peak": 100.0 * value / world / peak,
         "per_step_ms": {"step_median": per_step[0], "step_min": per_step[1],
-                        "prologue_median": per_step[2], "prologue_min": per_step[3],
-                        "attention_median": per_step[4], "attention_min": per_step[5]},
+                        "step_max": per_step[2], "prologue_median": per_step[3],
+                        "prologue_min": per_step[4], "attention_median": per_step[5],
+                        "attention_min": per_step[6], "attention_max": per_step[7]},
         "roofline": {
             "kernel": "packed_attention_kernel", "bound": "tensor", "achieved": att_tflops,
             "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak, "peak_kind": peak_kind,
