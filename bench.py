@@ -112,6 +112,15 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def wait_first_row(self, limit_s: float = 5.0):
+        """Block until nvidia-smi has written its first row (its start-up,
+        which can take a second, is then over before any timed work)."""
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < limit_s:
+            if os.path.getsize(self.path) > 0 or self.proc.poll() is not None:
+                return
+            time.sleep(0.02)
+
     def stop(self):
         if self.proc is None:
             return None
@@ -597,13 +606,14 @@ def main():
         if e2 is not None:
             e2.record(stream)
 
-    # The clock sampler starts before the warm-up (nvidia-smi needs a moment
-    # to come up), so that the timed region follows the warm-up with no idle
-    # gap in which the clocks could drop.
+    # The clock sampler is up (its first row written) before the warm-up, so
+    # that its start-up does not overlap the timed region and the timed
+    # region follows the warm-up with no idle gap in which the clocks could
+    # drop.
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if sampler:
         sampler.start()
-        time.sleep(0.3)
+        sampler.wait_first_row()
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()

@@ -199,7 +199,7 @@ extern "C" mf_status mf_qk_prologue_3d(const void* q, const void* k, const float
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int tok_per_block = mf::kPrologueThreads / (head_dim / 8);
+  const int tok_per_block = mf::kPrologueTokPerBlock;
   const unsigned grid = static_cast<unsigned>((total_tokens + tok_per_block - 1) / tok_per_block);
   if (head_dim == 128) {
     mf::qk_prologue_kernel<128><<<grid, mf::kPrologueThreads, 0, s>>>(

@@ -19,13 +19,15 @@
 // F = 0 is the 2D rotation above.
 //
 // HBM-bound: it reads q and k and writes q_hat and k_hat once (8 * T * H * d
-// bytes). Layout of the work: a group of d/8 threads owns one token and
-// loops over its heads; each thread holds 8 consecutive dims (one 16-byte vector) of q and of k, so a warp
-// reads and writes whole 256-byte rows, and it requests the next head's
-// vectors before it works on the current one. The token's position, gammas
-// and the 4 (cos, sin) pairs a thread needs are computed once per token
-// (theta of each pair once per block) and reused for all heads and for both
-// q and k.
+// bytes). Layout of the work: one warp owns one token and walks its heads in
+// groups of 32 / (d/8) (two heads at d = 128), each lane holding 8
+// consecutive dims (one 16-byte vector) of q and of k, so every load and
+// store instruction covers contiguous 512-byte spans. Each thread keeps the
+// next kPrologueDepth groups of its q and k in flight with cp.async into its
+// own shared-memory slots (no registers held, no barrier: a thread reads back
+// only what it copied). The token's position, gammas and (cos, sin) pairs
+// are computed once per token (theta of each pair once per block) and
+// reused for all heads and for both q and k.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -38,7 +40,8 @@
 
 namespace mf {
 
-// Threads per block of the backward's per-token kernels (delta, norm backward).
+// Threads per block of the per-token kernels (forward prologue, delta, norm
+// backward).
 constexpr int kPrologueThreads = 256;
 
 
@@ -135,6 +138,11 @@ __device__ __forceinline__ float2 pair_cos_sin(const TokenPos& tp, int pair, int
   return rotation_cos_sin(pos, pair_theta(e_in, width));
 }
 
+// Tokens of a forward prologue block: one per warp.
+constexpr int kPrologueTokPerBlock = kPrologueThreads / 32;
+// Head groups of q and k in flight per thread.
+constexpr int kPrologueDepth = 5;
+
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads, 4) qk_prologue_kernel(
     const uint4* __restrict__ q, const uint4* __restrict__ k, const float* __restrict__ gq_text,
@@ -142,25 +150,38 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) qk_prologue_kernel(
     const float* __restrict__ gk_img, const int32_t* __restrict__ cu_seqlens,
     const mf_segment* __restrict__ segs, int n_samples, int total_tokens, int heads, float eps,
     int frame_dims, uint4* __restrict__ q_hat, uint4* __restrict__ k_hat) {
-  constexpr int kVecPerRow = D / 8;  // 16-byte vectors per row
-  constexpr int kTokPerBlock = kPrologueThreads / kVecPerRow;
+  constexpr int kVecPerRow = D / 8;       // 16-byte vectors per row
+  constexpr int kRows = 32 / kVecPerRow;  // heads one warp instruction covers
+  constexpr int kP = kPrologueDepth;
   __shared__ double s_theta[D / 2];
   __shared__ int32_t s_axis[D / 2];
+  // Per thread: its 16 bytes of q and of k for kP head groups ahead.
+  __shared__ uint4 ring[kP][2][kPrologueThreads];
 
-  const int vec = threadIdx.x % kVecPerRow;
-  const int t_raw = blockIdx.x * kTokPerBlock + threadIdx.x / kVecPerRow;
-  // Threads past the last token compute on a valid token (so every lane of
-  // the warp takes part in the shuffles) and store nothing.
+  const int lane = threadIdx.x % 32;
+  const int vec = lane % kVecPerRow;
+  const int hsub = lane / kVecPerRow;  // head within each group of kRows
+  const int t_raw = blockIdx.x * kPrologueTokPerBlock + threadIdx.x / 32;
+  // A warp past the last token computes on a valid token and stores nothing.
   const bool active = t_raw < total_tokens;
   const int t = active ? t_raw : total_tokens - 1;
-  const size_t row0 = static_cast<size_t>(t) * heads * kVecPerRow + vec;
+  // Lane l holds vector l of the token's rows g*kRows .. g*kRows + kRows - 1:
+  // each instruction moves kRows * 2 * D contiguous bytes.
+  const size_t base = static_cast<size_t>(t) * heads * kVecPerRow + lane;
   const long long n_vec = static_cast<long long>(total_tokens) * heads * kVecPerRow;
+  const int n_groups = (heads + kRows - 1) / kRows;
 
-  // The first head's q and k are requested before any setup.
-  uint4 qv = make_uint4(0, 0, 0, 0), kv = make_uint4(0, 0, 0, 0);
-  if (in_bounds(row0, n_vec)) {
-    qv = __ldg(q + row0);
-    kv = __ldg(k + row0);
+  // The first kP groups are requested before any setup; every iteration
+  // commits one group of copies (empty past the end), so group g is always
+  // the (g+1)-th commit.
+#pragma unroll
+  for (int i = 0; i < kP; ++i) {
+    const size_t gi = base + static_cast<size_t>(i) * kRows * kVecPerRow;
+    if (i * kRows + hsub < heads && in_bounds(gi, n_vec)) {
+      cp_async16(&ring[i][0][threadIdx.x], q + gi);
+      cp_async16(&ring[i][1][threadIdx.x], k + gi);
+    }
+    cp_async_commit();
   }
   // theta and axis of every pair, once per block
   for (int pr = threadIdx.x; pr < D / 2; pr += kPrologueThreads) {
@@ -170,21 +191,31 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) qk_prologue_kernel(
   }
   __syncthreads();
 
-  // The token's position, gammas and the (cos, sin) of the 4 pairs this
-  // thread owns: once per token, for all its heads and for both q and k.
+  // The token's position, gammas and the (cos, sin) of the 4 pairs of a
+  // lane's 8 dims: once per token, for all heads and for both q and k. The
+  // kRows lanes that own the same dims compute 4 / kRows pairs each and swap.
   const TokenPos tp = token_position(cu_seqlens, segs, n_samples, t);
-  const int e0 = vec * 8;  // first dim this thread owns
+  const int e0 = vec * 8;  // first dim this lane owns
   float cs[4], sn[4];
+  {
+    float rc[4 / kRows], rs[4 / kRows];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int pair = e0 / 2 + i;
-    float2 r = make_float2(1.0f, 0.0f);
-    if (!tp.text) {
-      const int axis = s_axis[pair];
-      r = rotation_cos_sin(axis == 0 ? tp.frame : (axis == 1 ? tp.row : tp.col), s_theta[pair]);
+    for (int ii = 0; ii < 4 / kRows; ++ii) {
+      const int pair = e0 / 2 + ii * kRows + hsub;
+      float2 r = make_float2(1.0f, 0.0f);
+      if (!tp.text) {
+        const int axis = s_axis[pair];
+        r = rotation_cos_sin(axis == 0 ? tp.frame : (axis == 1 ? tp.row : tp.col), s_theta[pair]);
+      }
+      rc[ii] = r.x;
+      rs[ii] = r.y;
     }
-    cs[i] = r.x;
-    sn[i] = r.y;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int src = (i % kRows) * kVecPerRow + vec;
+      cs[i] = __shfl_sync(0xffffffffu, rc[i / kRows], src);
+      sn[i] = __shfl_sync(0xffffffffu, rs[i / kRows], src);
+    }
   }
   float gq[8], gk[8];
   {
@@ -198,18 +229,15 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) qk_prologue_kernel(
   }
 
   const float inv_d = 1.0f / D;
-#pragma unroll 2
-  for (int h = 0; h < heads; ++h) {
-    const size_t idx = row0 + static_cast<size_t>(h) * kVecPerRow;
-    // the next head's loads go out before this head's math
-    uint4 qn = make_uint4(0, 0, 0, 0), kn = make_uint4(0, 0, 0, 0);
-    if (h + 1 < heads) {
-      const size_t nidx = idx + kVecPerRow;
-      if (in_bounds(nidx, n_vec)) {
-        qn = __ldg(q + nidx);
-        kn = __ldg(k + nidx);
-      }
-    }
+  for (int g = 0; g < n_groups; ++g) {
+    const int h = g * kRows + hsub;
+    const bool head_in = h < heads;  // the last group may be partial
+    const size_t idx = base + static_cast<size_t>(g) * kRows * kVecPerRow;
+    const int slot = g % kP;
+    cp_async_wait<kP - 1>();  // group g has landed
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    const uint4 qv = head_in ? ring[slot][0][threadIdx.x] : zero;
+    const uint4 kv = head_in ? ring[slot][1][threadIdx.x] : zero;
     float xq[8], xk[8];
     unpack8(qv, xq);
     unpack8(kv, xk);
@@ -236,13 +264,20 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) qk_prologue_kernel(
       yk[2 * i] = ka * cs[i] - kb * sn[i];
       yk[2 * i + 1] = ka * sn[i] + kb * cs[i];
     }
-    if (active && in_bounds(idx, n_vec)) {
+    if (active && head_in && in_bounds(idx, n_vec)) {
       q_hat[idx] = pack8(yq);
       k_hat[idx] = pack8(yk);
     }
-    qv = qn;
-    kv = kn;
+    // The slot's values are in registers and used above: refill it with
+    // group g + kP.
+    const size_t gi = idx + static_cast<size_t>(kP) * kRows * kVecPerRow;
+    if (h + kP * kRows < heads && in_bounds(gi, n_vec)) {
+      cp_async16(&ring[slot][0][threadIdx.x], q + gi);
+      cp_async16(&ring[slot][1][threadIdx.x], k + gi);
+    }
+    cp_async_commit();
   }
+  cp_async_wait<0>();
 }
 
 }  // namespace mf
