@@ -153,11 +153,12 @@ template <int D>
 __device__ __forceinline__ void issue_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                              bool accumulate) {
   constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, D, 0, 1);
+  const uint32_t b_lo = lo32(b_desc);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    mma_ts(d_tmem, a_tmem + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
-           b_desc + static_cast<uint64_t>(kk * (2048 >> 4)), kIdesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_lo(d_tmem, a_tmem + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+              b_lo + static_cast<uint32_t>(kk * (2048 >> 4)), kIdesc,
+              (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D, bool kDq>
@@ -548,11 +549,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 template <int D>
 __device__ __forceinline__ void issue_rows_tmem(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc) {
   constexpr uint32_t kIdesc = idesc_bf16_f32(kSubM, kBlockN, 0, 0);
+  const uint32_t b_lo = lo32(b_desc);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8,
-           b_desc + static_cast<uint64_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4), kIdesc,
-           kk > 0 ? 1u : 0u);
+    mma_ts_lo(d_tmem, a_tmem + kk * 8,
+              b_lo + static_cast<uint32_t>(((kk / 4) * kBoxBytes + (kk % 4) * 32) >> 4), kIdesc,
+              kk > 0 ? 1u : 0u);
 }
 
 template <int D>
