@@ -84,6 +84,23 @@ def sample_rows(w: Workload, rng, n_random=256):
 @pytest.mark.parametrize("cfg,heads", [(0, None), (2, 2), (3, 1)])
 def test_prologue_matches_oracle(cuda_device, cfg, heads):
     w = WORKLOADS[cfg] if heads is None else WORKLOADS[cfg].with_heads(heads)
+    check_prologue(w, cuda_device)
+
+
+@pytest.mark.parametrize("d", (64, 128))
+@pytest.mark.parametrize("heads", (5, 11, 13, 22, 24))
+def test_prologue_head_groups(cuda_device, heads, d):
+    """A warp of the prologue covers 32 / (d/8) heads per instruction (2 at
+    d = 128, 4 at d = 64) and keeps five such groups in flight: head counts
+    whose last group is partial, with and without groups refilled beyond the
+    first five, on 74 tokens (a partial last block of 8 tokens)."""
+    w = Workload(f"heads{heads}_d{d}", ((13, 5, 7, 1), (0, 3, 4, 2), (1, 1, 1, 1)),
+                 heads=heads, head_dim=d, seed=90 + heads)
+    assert w.total_tokens == 74
+    check_prologue(w, cuda_device)
+
+
+def check_prologue(w: Workload, cuda_device):
     inp = make_inputs(w)
     plan = pa.PackedPlan(w.samples, w.heads, w.head_dim, w.token_budget, device=cuda_device)
     t = to_dev(inp, cuda_device)
