@@ -123,6 +123,8 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
             return None
         time.sleep(0.25)
         self.proc.terminate()

@@ -81,3 +81,48 @@ def test_reference_arm_line_and_non_zero_ranks():
                            "--config", "0", "--steps", "2", "--warmup", "1"],
                           capture_output=True, text=True, env=env1, timeout=120)
     assert out1.returncode == 0 and out1.stdout.strip() == ""
+
+
+def test_clock_sampler_waits_for_its_first_row_and_parses(monkeypatch, tmp_path):
+    """The sampler blocks until nvidia-smi has written a row (so its start-up
+    never overlaps timed work), then reports the median SM clock, the max
+    clock and every throttle reason seen. A stand-in for nvidia-smi writes
+    two rows after a delay."""
+    fake = tmp_path / "fake_smi.py"
+    fake.write_text(
+        "import sys, time\n"
+        "time.sleep(0.3)\n"
+        "print('0, 1965, 1965, 330.5, 0x0, Not Active, Not Active, Not Active, Not Active', flush=True)\n"
+        "print('0, 1800, 1965, 990.1, 0x4, Not Active, Not Active, Not Active, Active', flush=True)\n"
+        "time.sleep(30)\n")
+    real_popen = subprocess.Popen
+
+    def popen(args, **kw):
+        assert args[0] == "nvidia-smi" and "-lms" in args
+        return real_popen([sys.executable, str(fake)], **kw)
+
+    monkeypatch.setattr(bench.subprocess, "Popen", popen)
+    s = bench.ClockSampler(0)
+    s.start()
+    s.wait_first_row(limit_s=10.0)
+    assert os.path.getsize(s.path) > 0
+    clocks = s.stop()
+    assert clocks["samples"] == 2
+    assert clocks["sm_mhz"] == pytest.approx(1882.5)
+    assert clocks["sm_max_mhz"] == 1965.0
+    assert clocks["reasons"] == ["sw_power_cap"]
+    assert clocks["power_w_max"] == pytest.approx(990.1)
+
+
+def test_clock_sampler_without_nvidia_smi(monkeypatch):
+    """No nvidia-smi: the sampler reports nothing and never blocks."""
+    def popen(*a, **kw):
+        raise OSError("not found")
+
+    monkeypatch.setattr(bench.subprocess, "Popen", popen)
+    s = bench.ClockSampler(0)
+    s.start()
+    s.wait_first_row(limit_s=1.0)
+    path = s.path
+    assert s.stop() is None
+    assert not os.path.exists(path)  # its temporary file is removed too
