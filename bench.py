@@ -505,7 +505,8 @@ def report_all(args):
             "tokens_per_s": T / ((pro + att) / 1e3),
             "prologue_gbs": 8 * T * H * d / (pro / 1e3) / 1e9,
             "prologue_gbs_l2_flushed": 8 * T * H * d / (pro_flushed / 1e3) / 1e9,
-            "rope_frame_dims": w.rope_frame_dims, "peaks": peak_src}), flush=True)
+            "rope_frame_dims": w.rope_frame_dims, "peaks": peak_src,
+            "gpu": torch.cuda.get_device_name(dev)}), flush=True)
 
     # Training: forward with the log-normaliser, then the backward.
     for key, w in [(1, WORKLOADS[1]), (2, WORKLOADS[2]), (3, WORKLOADS[3]), (4, WORKLOADS[4]),
@@ -743,6 +744,7 @@ def main():
                        "across steps on three streams"},
         "gpu_launches": 2 * K,
         "clocks": clocks,
+        "gpu": torch.cuda.get_device_name(dev),
     }
     print(json.dumps(line), flush=True)
 
