@@ -94,3 +94,37 @@ def test_checked_build_reports_a_bad_sample_index(cuda_device):
         _, _, again = run_gpu(w, inp, cuda_device)
     _, _, ref = run_gpu(w, inp, cuda_device)
     assert torch.equal(again.view(torch.int16), ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("cfg", (1, 2, 3, 4))
+def test_checked_forward_full_size(cuda_device, cfg):
+    """The checked build on the full-size configs (every global index of the
+    prologue and the attention kernel compared with its buffer's extent at
+    the real sizes): no check fires, and the output is bit for bit the
+    product build's."""
+    from packed_attention_b200.workloads import WORKLOADS
+    w = WORKLOADS[cfg]
+    inp = make_inputs(w)
+    _, _, ref = run_gpu(w, inp, cuda_device)
+    with _native.checked_build():
+        _, _, got = run_gpu(w, inp, cuda_device)  # asserts no device error
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+
+
+def test_checked_backward_full_size(cuda_device):
+    """The checked build's backward on the full-size 1024² editing pack: no
+    check fires, and every gradient is bit for bit the product build's."""
+    from packed_attention_b200.workloads import WORKLOADS
+    w = WORKLOADS[3]
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    _, _, out_r, lse_r, g_r = run_fwd_bwd(w, inp, dob, cuda_device)
+    with _native.checked_build():
+        _, _, out_c, lse_c, g_c = run_fwd_bwd(w, inp, dob, cuda_device)  # asserts no error
+    assert torch.equal(out_c.view(torch.int16), out_r.view(torch.int16))
+    assert torch.equal(lse_c, lse_r)
+    for key in ("dq", "dk", "dv") + pa.GAMMA_NAMES:
+        a, b = g_c[key], g_r[key]
+        if a.dtype == torch.bfloat16:
+            a, b = a.view(torch.int16), b.view(torch.int16)
+        assert torch.equal(a, b), key
