@@ -224,6 +224,19 @@ def test_backward_random_packs(cuda_device, trial):
     check_grads(w.name, g, oracle_grads(w, inp, dob))
 
 
+def test_backward_many_small_samples(cuda_device):
+    """600 samples of 1 to ~100 tokens in one pack (one and two frames, 3D
+    rotation): every gradient within its bound, the four dgamma sums taken
+    over thousands of segment boundaries."""
+    rng = np.random.default_rng(1300)
+    samples = random_pack(rng, 600, 12, 7, 2)
+    w = Workload("bwd_many", samples, heads=2, head_dim=128, seed=1301, rope_frame_dims=16)
+    inp = make_inputs(w)
+    dob = dout_bits(w)
+    _, _, _, _, g = run_fwd_bwd(w, inp, dob, cuda_device)
+    check_grads(w.name, g, oracle_grads(w, inp, dob))
+
+
 def test_backward_uniform_512sq_all_heads(cuda_device):
     w = WORKLOADS[1]
     inp = make_inputs(w)

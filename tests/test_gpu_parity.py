@@ -182,6 +182,23 @@ def test_random_packs_full_compare(cuda_device, trial):
     assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
 
 
+@pytest.mark.parametrize("d", (64, 128))
+def test_many_small_samples_every_element(cuda_device, d):
+    """A pack of 600 samples of 1 to ~100 tokens (text only, grid only and
+    both; one and two frames), so that thousands of segment boundaries fall
+    inside warps, tiles and prologue blocks (600 work items per head): every
+    element against the oracle."""
+    rng = np.random.default_rng(9100 + d)
+    samples = random_pack(rng, 600, 12, 7, 2)
+    w = Workload(f"many_{d}", samples, heads=3, head_dim=d, seed=9200 + d)
+    assert len(w.seg_lens) == 600 and min(w.seg_lens) >= 1
+    inp = make_inputs(w)
+    _, _, out = run_gpu(w, inp, cuda_device)
+    ref = oracle.joint_attn(inp["q"], inp["k"], inp["v"], inp, w.samples, eps=w.eps)
+    max_abs, rel_rms = errors(bf16_to_f64(out), ref)
+    assert max_abs <= MAX_ABS and rel_rms <= REL_RMS, (max_abs, rel_rms)
+
+
 # ------------------------------------------------ full-size packs, sampled ---
 
 @pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
