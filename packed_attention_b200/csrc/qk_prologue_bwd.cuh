@@ -10,8 +10,8 @@
 //   dgamma += dy * x_n                    (per role q/k and modality)
 //   dx      = r * (dy * gamma - x_n * (x_n . (dy * gamma)) / d)
 //
-// Same layout of work as the forward prologue: d/8 threads own one token and
-// loop over its heads, 16-byte vectors; the token's rotation is set up once.
+// Layout of work: d/8 threads own one token and loop over its heads, 16-byte
+// vectors; the token's rotation is set up once.
 // The gamma gradients are reduced without atomics: per block in a fixed
 // order into a partial row, then over blocks in a fixed order, so that the
 // result is the same on every run.
